@@ -1,0 +1,397 @@
+"""Pins for the float64 oracle: closed forms, brute force on tiny inputs,
+library routines on the special cases that reduce to them, and the
+hand-derived fixtures in tests/golden/. CPU only."""
+
+import glob
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import sla_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(1234)
+
+
+def bits(x):
+    return W.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def head_from_blocks(blocks, N, pad):
+    """Expand per-block row cycles into an [N_pad, d] float32 array."""
+    Nb = len(blocks)
+    d = len(blocks[0][0])
+    x = np.empty((Nb * 64, d), dtype=np.float32)
+    for i, cyc in enumerate(blocks):
+        for t in range(64):
+            x[i * 64 + t] = cyc[t % len(cyc)]
+    x[N:] = pad
+    return x
+
+
+# ---------------------------------------------------------------------------
+# hand-derived fixtures
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path", sorted(glob.glob(os.path.join(GOLDEN, "*.json"))),
+                         ids=lambda p: os.path.basename(p))
+def test_golden_fixture(path):
+    g = json.load(open(path))
+    N = g["N"]
+    q, k, v = (head_from_blocks(g[t], N, g["pad"]) for t in ("q", "k", "v"))
+    kw = dict(variant=g["variant"], k_crit=g["k_crit"], k_neg=g["k_neg"])
+    if g["variant"] == "sla":
+        kw["w_proj_bits"] = bits(g["w_proj"])
+    else:
+        kw["alpha_h"] = g["alpha"]
+    r = O.forward_head(bits(q), bits(k), bits(v), N, **kw)
+    np.testing.assert_array_equal(r["Mc"], np.array(g["expected_Mc"], dtype=np.int8))
+    e = math.e
+    want = np.array([eval(x, {"e": e}) if isinstance(x, str) else x for x in g["expected_row"]])
+    np.testing.assert_allclose(r["O"], np.broadcast_to(want, r["O"].shape), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# phi
+# ---------------------------------------------------------------------------
+
+def test_phi_is_softmax_over_head_dim():
+    x = RNG.standard_normal((7, 5, 16)) * 3
+    p = O.phi(x)
+    assert np.all(p > 0)
+    np.testing.assert_allclose(p.sum(axis=-1), 1.0, atol=1e-14)
+    # invariant to a per-row shift, and ratios are exp of differences
+    np.testing.assert_allclose(O.phi(x + 11.5), p, atol=1e-15)
+    np.testing.assert_allclose(p[..., 3] / p[..., 9], np.exp(x[..., 3] - x[..., 9]), rtol=1e-12)
+    # large inputs stay finite (max-subtracted)
+    assert np.isfinite(O.phi(x * 1e3)).all()
+
+
+# ---------------------------------------------------------------------------
+# float32 specification of the mask scores
+# ---------------------------------------------------------------------------
+
+def test_pool_spec_exact_on_integers():
+    N = 64 * 5 + 23  # a partial last block of 23 rows
+    x = RNG.integers(-20, 21, size=(64 * 6, 8)).astype(np.float32)
+    got = O.pool_f32_spec(x, N)
+    exact = O.pool_f64(x.astype(np.float64), N)
+    # integer sums are exact in float32; full blocks divide by 64 exactly and the
+    # partial block by 23 with one rounding: at most half an ulp of float32
+    np.testing.assert_array_equal(got[:5], exact[:5].astype(np.float32))
+    ulp = np.spacing(np.abs(got[5]).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(got[5] - exact[5]) <= 0.5 * ulp + 1e-30)
+
+
+def test_pool_spec_close_to_mean_and_ignores_pad():
+    N = 64 * 3 + 10
+    x = RNG.standard_normal((64 * 4, 32)).astype(np.float32)
+    a = O.pool_f32_spec(x, N)
+    x2 = x.copy()
+    x2[N:] = np.nan
+    b = O.pool_f32_spec(x2, N)
+    np.testing.assert_array_equal(a, b)
+    ref = O.pool_f64(x.astype(np.float64), N)
+    assert np.abs(a - ref).max() < 64 * 2.0 ** -24 * 4
+
+
+def test_scores_and_router_spec_exact_on_small_integers():
+    qb = RNG.integers(-8, 9, size=(9, 16)).astype(np.float32)
+    kb = RNG.integers(-8, 9, size=(11, 16)).astype(np.float32)
+    Wt = RNG.integers(-4, 5, size=(16, 16)).astype(np.float32)
+    np.testing.assert_array_equal(O.scores_f32_spec(qb, kb), (qb.astype(np.float64) @ kb.T.astype(np.float64)))
+    np.testing.assert_array_equal(O.project_f32_spec(qb, Wt), qb.astype(np.float64) @ Wt.astype(np.float64))
+
+
+def test_scores_spec_is_sequential_float32_order():
+    # Non-integer case: the specified order accumulates k ascending from +0 with
+    # separately rounded products; check against a scalar loop on a few entries.
+    qb = RNG.standard_normal((4, 24)).astype(np.float32)
+    kb = RNG.standard_normal((5, 24)).astype(np.float32)
+    s = O.scores_f32_spec(qb, kb)
+    for i in range(4):
+        for j in range(5):
+            acc = np.float32(0.0)
+            for c in range(24):
+                acc = np.float32(acc + np.float32(qb[i, c] * kb[j, c]))
+            assert s[i, j] == acc
+
+
+# ---------------------------------------------------------------------------
+# classification
+# ---------------------------------------------------------------------------
+
+def brute_force_mask(s, kc, kn):
+    R, Nb = s.shape
+    Mc = np.zeros((R, Nb), dtype=np.int8)
+    for i in range(R):
+        for j in range(Nb):
+            rank = sum(1 for jj in range(Nb) if s[i, jj] > s[i, j] or (s[i, jj] == s[i, j] and jj < j))
+            if rank < kc:
+                Mc[i, j] = 1
+            elif rank >= Nb - kn:
+                Mc[i, j] = -1
+    return Mc
+
+
+@pytest.mark.parametrize("kc,kn", [(1, 0), (3, 2), (5, 11), (16, 0), (0, 4), (12, 4)])
+def test_classify_matches_rank_count_with_ties(kc, kn):
+    s = RNG.integers(-3, 4, size=(20, 16)).astype(np.float32)  # many ties
+    s[0] = 0.0
+    s[1, ::2] = -0.0  # signed zeros compare equal
+    Mc, crit, neg = O.classify(s, kc, kn)
+    np.testing.assert_array_equal(Mc, brute_force_mask(s, kc, kn))
+    for i in range(20):
+        assert list(crit[i]) == sorted(np.nonzero(Mc[i] == 1)[0])
+        assert list(neg[i]) == sorted(np.nonzero(Mc[i] == -1)[0])
+    # all-equal row: lowest indices critical, highest negligible
+    assert list(np.nonzero(Mc[0] == 1)[0]) == list(range(kc))
+    assert list(np.nonzero(Mc[0] == -1)[0]) == list(range(16 - kn, 16))
+
+
+def test_all_critical_and_constant_query():
+    s = RNG.standard_normal((6, 10)).astype(np.float32)
+    Mc, _, _ = O.classify(s, 10, 0)
+    assert np.all(Mc == 1)
+    s2 = np.broadcast_to(RNG.standard_normal(10).astype(np.float32), (6, 10))
+    Mc2, _, _ = O.classify(np.array(s2), 3, 2)
+    assert np.all(Mc2 == Mc2[0])
+
+
+def test_spec_mask_agrees_with_exact_ranking_on_tiny_workload():
+    w = W.WORKLOADS["sla_b1h2n1024d64"]
+    inp = W.make_inputs(w)
+    for h in range(w.H):
+        r = O.forward_head(inp.q[0, h], inp.k[0, h], inp.v[0, h], w.N, variant="sla",
+                           k_crit=w.k_crit, k_neg=w.k_neg, w_proj_bits=inp.w_proj,
+                           with_f64_mask=True)
+        for row, gaps in O.mask_disagreements(r, r["f64"], w.k_crit, w.k_neg):
+            assert min(gaps) < 1e-4, (row, gaps)
+
+
+def test_router_projection_commutes_with_pooling():
+    x = RNG.standard_normal((64 * 4, 16))
+    Wt = RNG.standard_normal((16, 16))
+    N = 64 * 3 + 5
+    np.testing.assert_allclose(O.pool_f64(x @ Wt, N), O.pool_f64(x, N) @ Wt, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# sparse branch
+# ---------------------------------------------------------------------------
+
+def rand_head(N, d, Np=None, scale=1.0):
+    Np = Np or 64 * ((N + 63) // 64)
+    x = (RNG.standard_normal((Np, d)) * scale).astype(np.float32)
+    return W.bf16_bits_to_f32(bits(x)).astype(np.float64)
+
+
+def test_sparse_all_critical_is_exact_softmax_attention():
+    import torch
+
+    N, d = 200, 16
+    q, k, v = rand_head(N, d, scale=2.0), rand_head(N, d, scale=2.0), rand_head(N, d)
+    Nb = q.shape[0] // 64
+    Mc = np.ones((Nb, Nb), dtype=np.int8)
+    scale = 1 / math.sqrt(d)
+    got = O.sparse_branch(q, k, v, Mc, N, scale)
+    # textbook dense softmax attention, full N x N
+    S = q[:N] @ k[:N].T * scale
+    P = np.exp(S - S.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(got, P @ v[:N], atol=1e-12)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a[:N]))[None, None]  # noqa: E731
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v))[0, 0].numpy()
+    np.testing.assert_allclose(got, ref, atol=1e-12)
+
+
+def test_sparse_branch_masks_exactly_the_noncritical_blocks():
+    N, d = 64 * 4, 8
+    q, k, v = rand_head(N, d), rand_head(N, d), rand_head(N, d)
+    Mc = np.array([[1, 0, -1, 1], [0, 0, 1, 0], [1, 1, 1, 1], [-1, 0, 0, 1]], dtype=np.int8)
+    got = O.sparse_branch(q, k, v, Mc, N, 0.3)
+    for r in range(N):
+        i = r // 64
+        keys = [t for t in range(N) if Mc[i, t // 64] == 1]
+        s = np.array([q[r] @ k[t] * 0.3 for t in keys])
+        p = np.exp(s - s.max())
+        want = (p[:, None] * v[keys]).sum(0) / p.sum()
+        np.testing.assert_allclose(got[r], want, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# linear branch
+# ---------------------------------------------------------------------------
+
+def brute_force_linear(q, k, v, Mc, N):
+    pq, pk = O.phi(q[:N]), O.phi(k[:N])
+    out = np.zeros((N, v.shape[1]))
+    for r in range(N):
+        i = r // 64
+        num = np.zeros(v.shape[1])
+        den = 0.0
+        for t in range(N):
+            if Mc[i, t // 64] == 0:
+                wgt = float(pq[r] @ pk[t])
+                num += wgt * v[t]
+                den += wgt
+        out[r] = num / den if den > 0 else 0.0
+    return out
+
+
+def test_linear_branch_matches_token_level_brute_force():
+    N, d = 64 * 3 + 17, 12
+    q, k, v = rand_head(N, d, scale=2), rand_head(N, d, scale=2), rand_head(N, d)
+    Mc = np.array([[1, 0, -1, 0], [0, 0, 0, 0], [1, 1, 1, 0], [-1, 1, 1, 1]], dtype=np.int8)
+    got = O.linear_branch(q, k, v, Mc, N)
+    np.testing.assert_allclose(got, brute_force_linear(q, k, v, Mc, N), atol=1e-12)
+    assert np.all(got[3 * 64:N] == 0.0)  # row 3 has no marginal block
+
+
+def test_no_critical_block_gives_pure_linear_attention():
+    # SLA with W = I and an empty critical set: O is linear attention over the
+    # non-negligible blocks; with k_neg = 0, over every token.
+    N, d = 64 * 4, 8
+    qb, kb, vb = bits(rand_head(N, d, scale=2)), bits(rand_head(N, d, scale=2)), bits(rand_head(N, d))
+    eye = bits(np.eye(d))
+    for kn in (0, 1):
+        r = O.forward_head(qb, kb, vb, N, variant="sla", k_crit=0, k_neg=kn, w_proj_bits=eye)
+        q, k, v = (W.bf16_bits_to_f32(b).astype(np.float64) for b in (qb, kb, vb))
+        np.testing.assert_allclose(r["O"], brute_force_linear(q, k, v, r["Mc"], N), atol=1e-12)
+        assert np.all(r["O_s"] == 0)
+    # k_neg = 0: every block marginal, plain linear attention over all tokens
+    pq, pk = O.phi(q), O.phi(k)
+    A = pq @ pk.T
+    r0 = O.forward_head(qb, kb, vb, N, variant="sla", k_crit=0, k_neg=0, w_proj_bits=eye)
+    np.testing.assert_allclose(r0["O"], (A @ v) / A.sum(1, keepdims=True), atol=1e-12)
+
+
+def test_sla2_alpha_extremes_and_empty_marginal():
+    N, d = 64 * 3, 16
+    qb, kb, vb = bits(rand_head(N, d, scale=2)), bits(rand_head(N, d, scale=2)), bits(rand_head(N, d))
+    full = O.forward_head(qb, kb, vb, N, variant="sla2", k_crit=3, k_neg=0, alpha_h=1.0)
+    q, k, v = (W.bf16_bits_to_f32(b).astype(np.float64) for b in (qb, kb, vb))
+    S = q @ k.T / math.sqrt(d)
+    P = np.exp(S - S.max(1, keepdims=True))
+    np.testing.assert_allclose(full["O"], (P / P.sum(1, keepdims=True)) @ v, atol=1e-12)
+    assert np.all(full["O_l"] == 0)  # no marginal block
+    zero = O.forward_head(qb, kb, vb, N, variant="sla2", k_crit=1, k_neg=0, alpha_h=0.0)
+    np.testing.assert_allclose(zero["O"], zero["O_l"], atol=0)
+
+
+def test_branch_outputs_are_convex_combinations_of_v():
+    w = W.WORKLOADS["sla_b1h2n1024d64"]
+    inp = W.make_inputs(w)
+    r = O.forward_head(inp.q[0, 0], inp.k[0, 0], inp.v[0, 0], w.N, variant="sla",
+                       k_crit=w.k_crit, k_neg=w.k_neg, w_proj_bits=inp.w_proj)
+    v = W.bf16_bits_to_f32(inp.v[0, 0])[:w.N].astype(np.float64)
+    for name, label in (("O_s", 1), ("O_l", 0)):
+        for i in range(w.Nb):
+            blocks = np.nonzero(r["Mc"][i] == label)[0]
+            rows = np.concatenate([v[j * 64:(j + 1) * 64] for j in blocks])
+            o = r[name][i * 64:(i + 1) * 64]
+            assert np.all(o <= rows.max(0) + 1e-12) and np.all(o >= rows.min(0) - 1e-12)
+
+
+def test_padding_rows_do_not_matter():
+    w = W.make_workload("pad", 1, 1, 64 * 5 + 9, 32, "sla", k_crit=2, k_neg=1, seed=9)
+    outs = []
+    for pad in (64.0, 0.0, float("nan"), -3e4):
+        inp = W.make_inputs(w.replace(pad_value=pad))
+        outs.append(O.forward(inp)[(0, 0)])
+    for o in outs[1:]:
+        np.testing.assert_array_equal(o["Mc"], outs[0]["Mc"])
+        np.testing.assert_array_equal(o["O"], outs[0]["O"])
+        assert np.isfinite(o["O"]).all()
+
+
+# ---------------------------------------------------------------------------
+# quantisation helpers
+# ---------------------------------------------------------------------------
+
+def e4m3_grid():
+    """All finite non-negative e4m3 values, from the format's definition."""
+    vals = [m * 2.0 ** -9 for m in range(8)]  # subnormals (exponent field 0)
+    for e in range(1, 16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue  # the NaN code
+            vals.append((1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(sorted(vals))
+
+
+def test_e4m3_round_is_nearest_even_on_the_grid():
+    grid = e4m3_grid()
+    assert grid[-1] == 448.0 and grid[8] == 2.0 ** -6
+    x = np.concatenate([RNG.standard_normal(20000) * 10.0 ** RNG.uniform(-4, 2.5, 20000), grid, -grid,
+                        (grid[1:] + grid[:-1]) / 2, [500.0, -1e6]])
+    y = O.e4m3_round(x)
+    a = np.abs(x)
+    assert np.all(np.isin(np.abs(y), grid))
+    # nearest: no grid point is strictly closer
+    idx = np.clip(np.searchsorted(grid, np.minimum(a, 448.0)), 1, grid.size - 1)
+    best = np.minimum(np.abs(grid[idx] - np.minimum(a, 448.0)), np.abs(grid[idx - 1] - np.minimum(a, 448.0)))
+    assert np.all(np.abs(np.abs(y) - np.minimum(a, 448.0)) <= best + 0.0)
+    assert np.all(np.abs(O.e4m3_round([500.0, -1e6])) == 448.0)
+    # ties go to the even code (mantissa lsb 0): 1 + 1/16 lies between 1 and 1.125
+    assert O.e4m3_round([1.0 + 1 / 16, 1.0 + 3 / 16])[0] == 1.0
+    assert O.e4m3_round([1.0 + 3 / 16])[0] == 1.25
+
+
+def test_e4m3_round_matches_torch_float8():
+    import torch
+
+    x = RNG.standard_normal(50000) * 10.0 ** RNG.uniform(-5, 2.6, 50000)
+    x = x[np.abs(x) <= 448.0].astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.e4m3_round(x.astype(np.float64)), ref)
+
+
+def test_int8_block_quantisation_bounds():
+    N = 64 * 2 + 30
+    x = (RNG.standard_normal((64 * 3, 16)) * 3).astype(np.float32)
+    codes, s = O.quantize_int8_blocks(x, N)
+    n = O.valid_rows(N, 3)
+    for i in range(3):
+        blk = x[i * 64:i * 64 + n[i]].astype(np.float64)
+        c = codes[i * 64:i * 64 + n[i]].astype(np.float64)
+        assert np.abs(c).max() == 127
+        assert np.all(np.abs(blk - c * s[i]) <= s[i] / 2 * (1 + 1e-6))
+    assert np.all(codes[N:] == 0)
+
+
+def test_quantized_branch_exact_when_inputs_sit_on_the_grids():
+    # Q, K integer-valued with block absmax 127 (INT8 scale exactly 1), keys
+    # equal inside each block (so P~ = 1 on the critical block), V on the e4m3
+    # grid with block absmax 448 (scale 1, r_j = 1): every quantisation step is
+    # exact and the emulated branch must equal the float64 sparse branch.
+    d, N = 8, 128
+    q = RNG.integers(-20, 21, size=(N, d)).astype(np.float32)
+    q[0, 0] = 127
+    q[64, 3] = -127
+    k = np.zeros((N, d), dtype=np.float32)
+    k[:64] = [127, 3, 0, 0, 0, 0, 0, 0]
+    k[64:] = [-127, 5, 1, 0, 0, 0, 0, 0]
+    grid = e4m3_grid()
+    v = (RNG.choice(grid[grid <= 448], size=(N, d)) * RNG.choice([-1, 1], size=(N, d))).astype(np.float32)
+    v[0, 0] = 448.0
+    v[64, 1] = -448.0
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    r = O.forward_head(qb, kb, vb, N, variant="sla2", k_crit=1, k_neg=0, alpha_h=1.0, quantized=True)
+    assert (r["Mc"] == 1).sum() == 2
+    np.testing.assert_allclose(r["O_sq"], r["O_s"], rtol=1e-13, atol=1e-12)
+
+
+def test_quantized_sparse_branch_error_is_quantisation_sized():
+    # Diagnostic scale only: on the tiny workload (128 critical keys per row)
+    # the low-bit branch stays within a few percent of the exact branch.
+    w = W.WORKLOADS["sla_b1h2n1024d64"]
+    inp = W.make_inputs(w)
+    r = O.forward_head(inp.q[0, 1], inp.k[0, 1], inp.v[0, 1], w.N, variant="sla",
+                       k_crit=w.k_crit, k_neg=w.k_neg, w_proj_bits=inp.w_proj, quantized=True)
+    err = r["O_sq"] - r["O_s"]
+    assert 0 < np.linalg.norm(err) / np.linalg.norm(r["O_s"]) < 0.1
