@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 SLA / SLA2 forward pass. Rank 0 prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one sla_forward over one batch of synthetic inputs (every stage of
+the forward: pooling, scores, classification, phi(K)/h/z, attention + linear +
+combine). The default workload is the SLA forward on a Wan2.1-1.3B-shaped call
+(B=1, H=12, N=32768, d=128, 5 % critical, 10 % negligible). value is
+dense-equivalent TFLOPS (full-attention FLOPs 4 B H N^2 d divided by the time,
+the pages' FLOPS definition). Inputs (3 x 100 MB) exceed the 126 MB L2, so no
+flush is needed between steps. With N > 1 (torchrun) every rank runs its own
+copy of the workload (independent heads: weak scaling, no data-path
+collective).
+
+--impl reference times the float64 CPU oracle (one head per step).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "sla_wan13b_b1h12n32768d128_s95"
+NORTH_STAR_97 = "sla2_b1h12n32768d128_s97"
+METRIC = "ms/forward and dense-equiv TFLOPS at 95-97% sparsity; tensor-pipe % of B200 peak"
+UNIT = "TFLOPS (dense-equivalent)"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# work accounting (algorithmic FLOPs / bytes; stated in the design doc)
+# ---------------------------------------------------------------------------
+
+def dense_eq_flops(w):
+    return 4.0 * w.B * w.H * w.N * w.N * w.d
+
+
+def attention_flops(w):
+    """Algorithmic tensor FLOPs of the attention kernel per launch: QK^T and PV on
+    every critical 64x64 pair, phi(Q) H for the linear branch, and (SLA) O^l W."""
+    BH = w.B * w.H
+    sparse = BH * w.Nb * w.k_crit * 4.0 * 64 * 64 * w.d
+    linear = BH * 2.0 * w.N * w.d * w.d
+    proj = BH * 2.0 * w.N * w.d * w.d if w.variant == "sla" else 0.0
+    return sparse + linear + proj
+
+
+def correction_flops(w):
+    """Extra tensor FLOPs executed for H_i = H_tot - sum over excluded blocks."""
+    return w.B * w.H * w.Nb * (w.k_crit + w.k_neg) * 4.0 * 64 * 64 * w.d
+
+
+def stage_bytes(w):
+    """Bytes each memory-bound stage moves (reads + writes) in this design."""
+    BH, N, Np, Nb, d = w.B * w.H, w.N, w.N_pad, w.Nb, w.d
+    nchunk = (Np + 1023) // 1024
+    return {
+        "pool": BH * (2 * N * d * 2 + 2 * Nb * d * 4),
+        "phik_hz": BH * (2 * N * d * 2 + Np * d * 2 + Nb * d * 4 + nchunk * d * d * 4),
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def device_inputs(inp):
+    import torch
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+    return dict(q=dev(inp.q), k=dev(inp.k), v=dev(inp.v),
+                w_proj=dev(inp.w_proj) if inp.w_proj is not None else None,
+                proj_q=dev(inp.proj_q) if inp.proj_q is not None else None,
+                proj_k=dev(inp.proj_k) if inp.proj_k is not None else None,
+                alpha=torch.from_numpy(inp.alpha).cuda() if inp.alpha is not None else None)
+
+
+def time_forward(sla, w, dev, steps, warmup, world, stage_timing=False, clocks=None):
+    """Device time of `steps` forwards (ms total, max over ranks) + per-stage ms."""
+    import torch
+
+    p = sla.make_params(w.B, w.H, w.N, w.d, variant=w.variant, k_crit=w.k_crit, k_neg=w.k_neg,
+                        w_proj=dev["w_proj"], proj_q=dev["proj_q"], proj_k=dev["proj_k"],
+                        alpha=dev["alpha"])
+    out = torch.empty_like(dev["q"])
+    ws = sla.allocate_workspace(p)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        sla.forward(dev["q"], dev["k"], dev["v"], out=out, workspace=ws, params=p, stream=stream)
+    torch.cuda.synchronize()
+    if stage_timing:
+        sla.stage_timing(steps)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    start.record(stream)
+    for _ in range(steps):
+        sla.forward(dev["q"], dev["k"], dev["v"], out=out, workspace=ws, params=p, stream=stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    ms = start.elapsed_time(end)
+    stages = None
+    if stage_timing:
+        stages, n = sla.stage_times()
+        sla.stage_timing(0)
+        stages = {k: v / max(n, 1) for k, v in stages.items()}
+    if sla.read_device_status(ws) != 0:
+        raise RuntimeError("device status reports a timeout")
+    return max_over_ranks(ms, world), stages, clk
+
+
+def time_dense(sla, w, dev, steps, warmup):
+    import torch
+
+    out = torch.empty_like(dev["q"])
+    for _ in range(warmup):
+        sla.dense_forward(dev["q"], dev["k"], dev["v"], N=w.N, out=out)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        sla.dense_forward(dev["q"], dev["k"], dev["v"], N=w.N, out=out)
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps
+
+
+def time_e2e(sla, w, inp, steps, warmup, world):
+    """Same metric through the C ABI with host buffers: each step copies Q, K, V
+    from pinned host memory, runs the forward and copies O back."""
+    import torch
+
+    def pinned(bits):
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory()
+
+    hq, hk, hv = pinned(inp.q), pinned(inp.k), pinned(inp.v)
+    ho = torch.empty_like(hq).pin_memory()
+    dev = device_inputs(inp)
+    q, k, v = dev["q"], dev["k"], dev["v"]
+    p = sla.make_params(w.B, w.H, w.N, w.d, variant=w.variant, k_crit=w.k_crit, k_neg=w.k_neg,
+                        w_proj=dev["w_proj"], proj_q=dev["proj_q"], proj_k=dev["proj_k"],
+                        alpha=dev["alpha"])
+    o = torch.empty_like(q)
+    ws = sla.allocate_workspace(p)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        sla.forward(q, k, v, out=o, workspace=ws, params=p, stream=stream)
+        ho.copy_(o, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end), world) / steps
+    nbytes = hq.numel() * 2
+    return ms, 3 * nbytes, nbytes
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """The float64 oracle, as it stands, on a bounded sample of heads of the workload."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import sla_oracle as O
+
+    heads = [(0, h) for h in range(w.H)]
+    t0 = time.perf_counter()
+    done = 0
+    for bh in heads:
+        inp = W.make_inputs(w, heads=[bh])
+        t = time.perf_counter()
+        O.forward(inp)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    elapsed = time.perf_counter() - t0
+    flops = 4.0 * w.N * w.N * w.d * done
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": flops / elapsed / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {w.B * w.H} heads of {w.name}, every query block, float64 NumPy "
+                      f"(input generation included), {elapsed:.1f} s"}
+
+
+def run_ours(args):
+    import torch
+
+    import sparse_linear_attention_pool_b200 as sla
+
+    world, rank, local = dist_setup(args.gpus)
+    sla.load()
+    pk, pk_kind = peaks()
+    w = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(w)
+    dev = device_inputs(inp)
+    clocks = ClockSampler(local)
+    ms_total, stages, clk = time_forward(sla, w, dev, args.steps, args.warmup, world,
+                                         stage_timing=True, clocks=clocks)
+    ms = ms_total / args.steps
+    value = dense_eq_flops(w) * world / (ms * 1e-3) / 1e12
+
+    # dominant kernel: the attention stage (tensor cores)
+    attn_ms = stages["attention"]
+    attn_alg = attention_flops(w)
+    attn_tf = attn_alg / (attn_ms * 1e-3) / 1e12
+    peak_tf = pk["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4), "traffic": None,
+                "kernel": "attention", "peak_kind": f"{pk_kind} bf16 sustained",
+                "executed_tflops_incl_correction":
+                    round((attn_alg + correction_flops(w)) / (attn_ms * 1e-3) / 1e12, 2)}
+    sb = stage_bytes(w)
+    hbm = {k: {"ms": round(stages[k], 4), "GB/s": round(b / (stages[k] * 1e-3) / 1e9, 1),
+               "frac": round(b / (stages[k] * 1e-3) / 1e9 / pk["hbm_gbs"], 4), "bytes": b}
+           for k, b in sb.items()}
+
+    res = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded block-clustered Q/K, Gaussian V; Wan2.1-shaped)",
+           "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                      "variant": w.variant, "k_crit": w.k_crit, "k_neg": w.k_neg,
+                      "sparsity": round(w.sparsity, 4), "global_batch": w.B * world,
+                      "seq_len": w.N, "parallelism": f"independent replicas x{world}",
+                      "l2": "inputs (302 MB) larger than L2; no flush"},
+           "roofline": roofline,
+           "stages_ms": {k: round(v, 4) for k, v in stages.items()},
+           "hbm_stages": hbm,
+           "gpu_launches": 6 * args.steps,
+           "clocks": clk}
+
+    if not args.no_dense and rank == 0:
+        dense_ms = time_dense(sla, w, dev, args.dense_steps, 2)
+        res["dense_baseline"] = {"ms": round(dense_ms, 4),
+                                 "tflops": round(dense_eq_flops(w) / (dense_ms * 1e-3) / 1e12, 2),
+                                 "speedup_of_sparse": round(dense_ms / ms, 3)}
+    if not args.no_north_star and rank == 0 and args.workload != NORTH_STAR_97:
+        w97 = W.WORKLOADS[NORTH_STAR_97]
+        inp97 = W.make_inputs(w97)
+        dev97 = device_inputs(inp97)
+        ms97, st97, _ = time_forward(sla, w97, dev97, args.steps, args.warmup, 1, stage_timing=True)
+        ms97 /= args.steps
+        entry = {"workload": w97.name, "ms": round(ms97, 4),
+                 "dense_eq_tflops": round(dense_eq_flops(w97) / (ms97 * 1e-3) / 1e12, 2),
+                 "attention_ms": round(st97["attention"], 4),
+                 "attention_tflops": round(attention_flops(w97) / (st97["attention"] * 1e-3) / 1e12, 2)}
+        if "dense_baseline" in res:
+            entry["speedup_vs_dense"] = round(res["dense_baseline"]["ms"] / ms97, 3)
+        res["north_star_97"] = entry
+        del dev97
+    if not args.no_e2e:
+        e_ms, h2d, d2h = time_e2e(sla, w, inp, max(3, args.steps // 4), 2, world)
+        res["e2e"] = {"value": round(dense_eq_flops(w) * world / (e_ms * 1e-3) / 1e12, 3),
+                      "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "ms_per_step": round(e_ms, 4)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as it stands, timed on the host cores: one head per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_info
+
+    from oracle import sla_oracle as O
+
+    w = W.WORKLOADS[args.workload]
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    samples = [W.make_inputs(w, heads=[heads[i % len(heads)]]) for i in range(min(len(heads), 4))]
+    for i in range(args.warmup):
+        O.forward(samples[i % len(samples)])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        O.forward(samples[i % len(samples)])
+    sec = (time.perf_counter() - t0) / args.steps
+    value = 4.0 * w.N * w.N * w.d / sec / 1e12
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    res = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(sec * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                      "variant": w.variant, "k_crit": w.k_crit, "k_neg": w.k_neg},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                            "sample": f"one head of {w.name} per step (every query block), "
+                                      "float64 NumPy"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--dense-steps", type=int, default=5)
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-north-star", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

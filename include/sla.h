@@ -1,0 +1,174 @@
+/*
+ * sla.h -- C ABI of the B200 (sm_100a) SLA / SLA2 sparse-linear attention forward pass.
+ *
+ * One call, sla_forward(), runs the whole forward of a batch of heads on one
+ * GPU, every step in this library's CUDA kernels:
+ *
+ *   1. block mean pooling of Q and K over 64-token blocks (SLA2: followed by the
+ *      learnable router projections proj_q / proj_k);
+ *   2. pooled scores s_ij = qbar_i . kbar_j and the per-row three-way block
+ *      classification into the compressed mask Mc (1 critical, 0 marginal,
+ *      -1 negligible) plus the ascending index lists of critical / negligible
+ *      blocks;
+ *   3. phi(K) (softmax over the head dimension) and the linear-attention sums
+ *      h_j = phi(K_j)^T V_j, z_j = rowsum(phi(K_j)^T);
+ *   4. per 64-row query block: softmax attention over the critical key blocks
+ *      (online softmax, tensor cores), the linear branch
+ *      phi(Q_i) H_i / phi(Q_i) Z_i over the marginal blocks, and the combine
+ *      (SLA: O = O^s + O^l W; SLA2: O = alpha_h O^s + (1 - alpha_h) O^l).
+ *
+ * Sources (page title, section):
+ *   - "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable
+ *     Sparse-Linear Attention", structured summary (aipaper.cc), section 4
+ *     "Methodology": formula 1 (Pc from pooled Q, K), formula 2 (Mc), formula 3
+ *     (H_i, Z_i, O^l_i), formula 4 (O = O^s + Proj(O^l)).
+ *   - SLA walkthrough (intelliparadigm.com), sections 1.2 and 2.2: bq = bkv = 64,
+ *     precomputed h_j / z_j, online softmax, one fused kernel; section 3.2:
+ *     phi = softmax.
+ *   - SLA2 article, arXiv 2602.12675 (mcffsbgs.com): O = alpha O^s +
+ *     (1 - alpha) O^l, router with two projection matrices, low-bit Q, K, P, V.
+ *   - "SLA2 -- L3 Cross-Paper Synthesis" (zhaifeiyue.github.io), section 2:
+ *     alpha mixing replaces SLA's projection; router proj_q / proj_k.
+ *
+ * Conventions
+ *   - Q, K, V, O: contiguous row-major [B, H, N_pad, d] bfloat16 in device
+ *     memory, N_pad = 64 * ceil(N / 64). Rows N .. N_pad-1 of Q, K, V are pad:
+ *     never read into any result (they may hold anything, NaN included).
+ *     Rows N .. N_pad-1 of O are not written. Base addresses 16-byte aligned.
+ *   - d is 64 or 128. Block sizes are fixed at 64 x 64.
+ *   - Every call is asynchronous on the given stream (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream) and enqueues only kernels,
+ *     cudaMemsetAsync and cudaMemcpyAsync. The library never allocates or frees
+ *     memory and never synchronises, except sla_read_device_status().
+ *   - Ownership: the caller owns every buffer (inputs, outputs, weights and the
+ *     workspace) and must keep them alive until the stream work completes.
+ *   - Errors are returned as sla_status codes; arguments are validated before
+ *     anything is enqueued, so a non-SLA_OK return from validation means
+ *     nothing ran. SLA_ERR_CUDA reports a launch or runtime error.
+ *   - Reentrancy: calls may run concurrently on different streams if each uses
+ *     its own workspace. Results are deterministic: the same inputs give
+ *     bitwise identical O, Mc and index lists (no floating-point atomics).
+ */
+#ifndef SLA_H_
+#define SLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SLA_ABI_VERSION 1
+#define SLA_BLOCK 64
+#define SLA_MAX_BLOCKS 4096 /* N <= 262144 */
+
+typedef enum {
+  SLA_OK = 0,
+  SLA_ERR_INVALID_ARG = 1,    /* a null pointer, a bad size or count, a bad enum value */
+  SLA_ERR_UNSUPPORTED = 2,    /* valid request this build does not implement (e.g. d not 64/128) */
+  SLA_ERR_WORKSPACE = 3,      /* workspace missing, misaligned (256 B) or smaller than required */
+  SLA_ERR_ALIGNMENT = 4,      /* a tensor base address not 16-byte aligned */
+  SLA_ERR_CUDA = 5,           /* a CUDA launch or runtime call failed */
+  SLA_ERR_DEVICE_TIMEOUT = 6, /* a bounded wait inside a kernel expired (see sla_read_device_status) */
+  SLA_ERR_DEVICE_CHECK = 7    /* an in-kernel consistency check failed (e.g. a block index out of range) */
+} sla_status;
+
+typedef enum { SLA_VARIANT_SLA = 0, SLA_VARIANT_SLA2 = 1 } sla_variant;
+
+typedef enum {
+  SLA_PREC_BF16 = 0,      /* bf16 tensor-core products, fp32 accumulation */
+  SLA_PREC_I8QK_F8PV = 1  /* sparse branch with INT8 Q K^T and FP8 e4m3 P V */
+} sla_precision;
+
+typedef struct sla_params {
+  int B, H;            /* batch and heads (>= 1) */
+  int N;               /* true sequence length (>= 1); tensors hold N_pad rows */
+  int d;               /* head dimension: 64 or 128 */
+  int block_q;         /* must be 64 */
+  int block_kv;        /* must be 64 */
+  int variant;         /* sla_variant */
+  int precision;       /* sla_precision */
+  int k_crit;          /* critical blocks per row: 1 <= k_crit <= Nb */
+  int k_neg;           /* negligible blocks per row: 0 <= k_neg, k_crit + k_neg <= Nb */
+  float softmax_scale; /* scale of q.k in the sparse branch; 0 selects 1/sqrt(d) */
+  const void* w_proj;  /* SLA: [d, d] bf16 device, y = x W (row-major [in][out]); NULL = identity */
+  const void* proj_q;  /* SLA2 router: [d, d] bf16 device, qbar W_q; NULL = none (both or neither) */
+  const void* proj_k;  /* SLA2 router: [d, d] bf16 device, kbar W_k */
+  const float* alpha;  /* SLA2: [H] float32 device, per-head mixing weight; required for SLA2 */
+} sla_params;
+
+/* ABI version of the loaded library (SLA_ABI_VERSION at build time). */
+int sla_abi_version(void);
+
+/* Static description of a status code; never NULL. */
+const char* sla_status_string(sla_status status);
+
+/* Bytes of device workspace sla_forward() needs for these parameters, or 0 if
+ * the parameters are invalid (call sla_validate for the reason). */
+size_t sla_workspace_size(const sla_params* p);
+
+/* Checks the parameters alone (no pointers to tensors): SLA_OK or the error
+ * sla_forward would return for them. */
+sla_status sla_validate(const sla_params* p);
+
+/* The forward pass (steps 1-4 above).
+ *   Q, K, V   [B, H, N_pad, d] bf16 device inputs.
+ *   O         [B, H, N_pad, d] bf16 device output (rows >= N untouched).
+ *   workspace device scratch of at least sla_workspace_size(p) bytes,
+ *             256-byte aligned; its contents on entry do not matter. After the
+ *             call it holds the pooled vectors, Mc and the index lists
+ *             (read them with sla_get_mask / sla_get_pooled) until reused.
+ *   stream    cudaStream_t as void*. */
+sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, const sla_params* p,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Copies the compressed mask and block lists of the last sla_forward() that
+ * used this workspace (stream-ordered, device to device; any output may be NULL).
+ *   mc    [B, H, Nb, Nb] int8: 1 critical, 0 marginal, -1 negligible.
+ *   crit  [B, H, Nb, k_crit] int32, ascending block indices.
+ *   neg   [B, H, Nb, k_neg] int32, ascending block indices. */
+sla_status sla_get_mask(const sla_params* p, const void* workspace, int8_t* mc, int32_t* crit,
+                        int32_t* neg, void* stream);
+
+/* Copies the pooled (SLA2: pooled and router-projected) vectors the mask was
+ * ranked on, [B, H, Nb, d] float32 each (device to device; either may be NULL). */
+sla_status sla_get_pooled(const sla_params* p, const void* workspace, float* qbar, float* kbar,
+                          void* stream);
+
+/* Synchronises the stream, then reads the device status word written by the
+ * last sla_forward() on this workspace: SLA_OK, SLA_ERR_DEVICE_TIMEOUT if a
+ * bounded in-kernel wait gave up, or SLA_ERR_DEVICE_CHECK if an in-kernel check
+ * failed (in both cases the output is not valid). */
+sla_status sla_read_device_status(const void* workspace, void* stream);
+
+/* Dense softmax attention O = softmax(Q K^T * scale) V over all N keys, with
+ * the same kernel machinery as the sparse branch (every block critical, no
+ * linear branch, no mask). The baseline the pages compare against
+ * (FlashAttention, SLA structured summary section 6, kernel-speed figure).
+ * Same tensor layout as sla_forward; no workspace. */
+sla_status sla_dense_forward(const void* Q, const void* K, const void* V, void* O, int B, int H,
+                             int N, int d, float softmax_scale, void* stream);
+
+/* Stage timing, a profiling aid (no counterpart on the pages). Stages of
+ * sla_forward, in order: 0 pooling (+ router), 1 pooled scores, 2 classification,
+ * 3 phi(K) / z_j / partial H, 4 H_tot / Z_tot reduction, 5 attention (sparse +
+ * linear + combine). */
+#define SLA_NUM_STAGES 6
+
+/* max_calls > 0: create CUDA events (on the current device) for up to max_calls
+ * sla_forward calls and start recording: each call records an event before its
+ * first stage and after every stage, on its stream. 0: stop and release the
+ * events. Process-wide state, not thread-safe; off by default. */
+sla_status sla_stage_timing(int max_calls);
+
+/* Waits for the recorded events, writes the summed elapsed milliseconds of each
+ * stage over the recorded calls to ms[SLA_NUM_STAGES] and their number to
+ * *calls, then clears the record (recording continues). */
+sla_status sla_stage_times(float* ms, int* calls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H_ */

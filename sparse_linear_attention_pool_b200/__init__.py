@@ -1,0 +1,218 @@
+"""Python binding of the B200 SLA / SLA2 forward-pass library (libsla_b200.so).
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels. PyTorch supplies device memory and the stream. There is no CPU
+fallback: if the compiled library is missing, load() raises.
+
+    import sparse_linear_attention_pool_b200 as sla
+    o = sla.forward(q, k, v, N=N, variant="sla2", k_crit=15, alpha=alpha,
+                    proj_q=wq, proj_k=wk)
+
+q, k, v: [B, H, N_pad, d] torch.bfloat16 CUDA tensors, N_pad = 64 * ceil(N / 64).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsla_b200.so")
+
+SLA_OK, SLA_ERR_INVALID_ARG, SLA_ERR_UNSUPPORTED, SLA_ERR_WORKSPACE, SLA_ERR_ALIGNMENT, \
+    SLA_ERR_CUDA, SLA_ERR_DEVICE_TIMEOUT, SLA_ERR_DEVICE_CHECK = range(8)
+VARIANTS = {"sla": 0, "sla2": 1}
+PRECISIONS = {"bf16": 0, "i8qk_f8pv": 1}
+BLOCK = 64
+
+# every symbol include/sla.h declares
+EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate", "sla_workspace_size",
+           "sla_forward", "sla_get_mask", "sla_get_pooled", "sla_read_device_status",
+           "sla_dense_forward", "sla_stage_timing", "sla_stage_times")
+NUM_STAGES = 6
+STAGES = ("pool", "scores", "classify", "phik_hz", "hz_reduce", "attention")
+
+
+class Params(ctypes.Structure):
+    """Mirror of struct sla_params."""
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
+        ("block_q", ctypes.c_int), ("block_kv", ctypes.c_int),
+        ("variant", ctypes.c_int), ("precision", ctypes.c_int),
+        ("k_crit", ctypes.c_int), ("k_neg", ctypes.c_int),
+        ("softmax_scale", ctypes.c_float),
+        ("w_proj", ctypes.c_void_p), ("proj_q", ctypes.c_void_p), ("proj_k", ctypes.c_void_p),
+        ("alpha", ctypes.c_void_p),
+    ]
+
+
+class SLAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the compiled library (once). Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} not built; run python -m sparse_linear_attention_pool_b200.build")
+    lib = ctypes.CDLL(path)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    P = ctypes.POINTER(Params)
+    sig = {
+        "sla_abi_version": (i, []),
+        "sla_status_string": (ctypes.c_char_p, [i]),
+        "sla_validate": (i, [P]),
+        "sla_workspace_size": (sz, [P]),
+        "sla_forward": (i, [vp, vp, vp, vp, P, vp, sz, vp]),
+        "sla_get_mask": (i, [P, vp, vp, vp, vp, vp]),
+        "sla_get_pooled": (i, [P, vp, vp, vp, vp]),
+        "sla_read_device_status": (i, [vp, vp]),
+        "sla_dense_forward": (i, [vp, vp, vp, vp, i, i, i, i, ctypes.c_float, vp]),
+        "sla_stage_timing": (i, [i]),
+        "sla_stage_times": (i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().sla_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != SLA_OK:
+        raise SLAError(status, what)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_params(B, H, N, d, *, variant="sla", precision="bf16", k_crit, k_neg=0,
+                softmax_scale=0.0, w_proj=None, proj_q=None, proj_k=None, alpha=None) -> Params:
+    return Params(B=B, H=H, N=N, d=d, block_q=BLOCK, block_kv=BLOCK,
+                  variant=VARIANTS[variant], precision=PRECISIONS[precision],
+                  k_crit=int(k_crit), k_neg=int(k_neg), softmax_scale=float(softmax_scale),
+                  w_proj=_ptr(w_proj), proj_q=_ptr(proj_q), proj_k=_ptr(proj_k), alpha=_ptr(alpha))
+
+
+def validate(p: Params) -> int:
+    return load().sla_validate(ctypes.byref(p))
+
+
+def workspace_size(p: Params) -> int:
+    n = load().sla_workspace_size(ctypes.byref(p))
+    if n == 0:
+        _check(validate(p), "sla_workspace_size")
+    return n
+
+
+def allocate_workspace(p: Params, device=None):
+    """A uint8 CUDA tensor of sla_workspace_size bytes (torch allocations are 256-aligned)."""
+    import torch
+
+    return torch.empty(workspace_size(p), dtype=torch.uint8, device=device or "cuda")
+
+
+def forward(q, k, v, *, N: Optional[int] = None, variant: str = "sla", precision: str = "bf16",
+            k_crit: Optional[int] = None, k_neg: int = 0, softmax_scale: float = 0.0, w_proj=None,
+            proj_q=None, proj_k=None, alpha=None, out=None, workspace=None, stream=None,
+            params=None):
+    """O = SLA / SLA2 forward of q, k, v ([B, H, N_pad, d] bf16 CUDA tensors).
+
+    Returns (O, workspace); the workspace holds the mask and lists afterwards."""
+    import torch
+
+    B, H, Np, d = q.shape
+    N = Np if N is None else int(N)
+    if params is None and k_crit is None:
+        raise ValueError("forward() needs k_crit or params")
+    p = params or make_params(B, H, N, d, variant=variant, precision=precision, k_crit=k_crit,
+                              k_neg=k_neg, softmax_scale=softmax_scale, w_proj=w_proj,
+                              proj_q=proj_q, proj_k=proj_k, alpha=alpha)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = allocate_workspace(p, q.device)
+    st = load().sla_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(p),
+                            _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sla_forward")
+    return out, workspace
+
+
+def get_mask(p: Params, workspace, stream=None):
+    """(Mc [B,H,Nb,Nb] int8, crit [B,H,Nb,kc] int32, neg [B,H,Nb,kn] int32) on the device."""
+    import torch
+
+    Nb = (p.N + BLOCK - 1) // BLOCK
+    dev = workspace.device
+    mc = torch.empty((p.B, p.H, Nb, Nb), dtype=torch.int8, device=dev)
+    crit = torch.empty((p.B, p.H, Nb, p.k_crit), dtype=torch.int32, device=dev)
+    neg = torch.empty((p.B, p.H, Nb, p.k_neg), dtype=torch.int32, device=dev)
+    st = load().sla_get_mask(ctypes.byref(p), _ptr(workspace), _ptr(mc), _ptr(crit),
+                             _ptr(neg) if p.k_neg > 0 else None, _stream(stream))
+    _check(st, "sla_get_mask")
+    return mc, crit, neg
+
+
+def get_pooled(p: Params, workspace, stream=None):
+    """(qbar, kbar) [B,H,Nb,d] float32: the vectors the mask was ranked on."""
+    import torch
+
+    Nb = (p.N + BLOCK - 1) // BLOCK
+    qb = torch.empty((p.B, p.H, Nb, p.d), dtype=torch.float32, device=workspace.device)
+    kb = torch.empty_like(qb)
+    _check(load().sla_get_pooled(ctypes.byref(p), _ptr(workspace), _ptr(qb), _ptr(kb),
+                                 _stream(stream)), "sla_get_pooled")
+    return qb, kb
+
+
+def read_device_status(workspace, stream=None) -> int:
+    return load().sla_read_device_status(_ptr(workspace), _stream(stream))
+
+
+def dense_forward(q, k, v, *, N: Optional[int] = None, softmax_scale: float = 0.0, out=None,
+                  stream=None):
+    """Dense softmax attention with the same kernel machinery (the baseline)."""
+    import torch
+
+    B, H, Np, d = q.shape
+    N = Np if N is None else int(N)
+    if out is None:
+        out = torch.empty_like(q)
+    st = load().sla_dense_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d,
+                                  float(softmax_scale), _stream(stream))
+    _check(st, "sla_dense_forward")
+    return out
+
+
+def stage_timing(max_calls: int):
+    """Record per-stage CUDA events for up to max_calls sla_forward calls (0 stops)."""
+    _check(load().sla_stage_timing(int(max_calls)), "sla_stage_timing")
+
+
+def stage_times() -> tuple[dict, int]:
+    """(summed ms per stage name, number of calls) since the last read."""
+    ms = (ctypes.c_float * NUM_STAGES)()
+    n = ctypes.c_int(0)
+    _check(load().sla_stage_times(ms, ctypes.byref(n)), "sla_stage_times")
+    return {name: float(ms[i]) for i, name in enumerate(STAGES)}, n.value

@@ -1,0 +1,184 @@
+// Linear-attention precompute (step 3 of the forward): phi(K) with
+// phi = softmax over the head dimension, the per-block column sums
+// z_j = rowsum(phi(K_j)^T), and the per-head totals
+// H_tot = sum_j phi(K_j)^T V_j, Z_tot = sum_j z_j.
+//
+// Source: SLA walkthrough (intelliparadigm.com), section 1.2 ("precompute
+// h_j = phi(K_j)^T V_j and z_j = rowsum(phi(K_j)^T)") and section 2.2
+// (the H / Z accumulation pseudo-code); SLA structured summary (aipaper.cc),
+// section 4, formula 3; phi = softmax: walkthrough section 3.2.
+//
+// The per-query-block sums over marginal blocks are formed later as
+// H_i = H_tot - sum_{j excluded from row i} h_j (likewise Z_i), with the
+// excluded (critical and negligible) blocks' terms recomputed from the tiles
+// the attention kernel loads, so H_tot / Z_tot are all that is stored here.
+// Reductions run in a fixed order (no atomics): results are deterministic.
+#include "sla_internal.cuh"
+
+namespace sla {
+
+// CTA of 256 threads (8 warps) per (1024-token chunk, head). For each 64-token
+// block: phi(K) rows -> global (bf16) and shared memory, z_j -> global,
+// H_chunk += phi(K_j)^T V_j on tensor cores (mma.sync m16n8k16, fp32 acc).
+template <int D>
+__global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __restrict__ K,
+                                                      const __nv_bfloat16* __restrict__ V,
+                                                      __nv_bfloat16* __restrict__ phik,
+                                                      float* __restrict__ zblk,
+                                                      float* __restrict__ hpart, int N, int Npad,
+                                                      int Nb, int nchunk) {
+  constexpr int CPR = D / 8;            // 16-byte chunks per row
+  constexpr int WPM = 128 / D;          // warps per 16-row m tile (1 for D=128, 2 for D=64)
+  constexpr int NCOL = D / WPM;         // output columns per warp
+  constexpr int NT = NCOL / 8;          // n tiles per warp
+  __shared__ __align__(128) __nv_bfloat16 PK[64 * D];
+  __shared__ __align__(128) __nv_bfloat16 Vs[64 * D];
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = warp / WPM, n0 = (warp % WPM) * NCOL;
+  const size_t hoff = size_t(bh) * Npad * D;
+  const int jb0 = chunk * (kHzChunk / kBlock);
+  const int jb1 = min(Nb, jb0 + kHzChunk / kBlock);
+
+  float acc[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[t][e] = 0.0f;
+
+  for (int jb = jb0; jb < jb1; ++jb) {
+    const int t0 = jb * kBlock;
+    const int nv = min(kBlock, N - t0);
+    // V tile (rows >= N zero-filled)
+    for (int id = threadIdx.x; id < 64 * CPR; id += 256) {
+      const int r = id / CPR, ch = id % CPR;
+      const bool v = r < nv;
+      cp_async16(smem_u32(Vs + r * D + ((ch ^ (r & 7)) << 3)),
+                 v ? (const void*)(V + hoff + size_t(t0 + r) * D + ch * 8) : (const void*)V, v);
+    }
+    cp_async_commit();
+    // phi(K) rows: warp w handles rows w, w+8, ...; a lane holds D/32 columns
+    for (int r = warp; r < 64; r += 8) {
+      constexpr int PL = D / 32;
+      float x[PL];
+      const int col = lane * PL;
+      __nv_bfloat16* gdst = phik + hoff + size_t(t0 + r) * D + col;
+      if (r < nv) {
+        const __nv_bfloat16* src = K + hoff + size_t(t0 + r) * D + col;
+        float m = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) {
+          x[e] = bf2f(src[e]);
+          m = fmaxf(m, x[e]);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float s = 0.0f;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) {
+          x[e] = expf(x[e] - m);
+          s += x[e];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        const float inv = 1.0f / s;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) x[e] *= inv;
+      } else {
+#pragma unroll
+        for (int e = 0; e < PL; ++e) x[e] = 0.0f;
+      }
+      uint32_t pk[PL / 2];
+#pragma unroll
+      for (int e = 0; e < PL / 2; ++e) pk[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+      __nv_bfloat16* sdst = PK + swz(r, col, D);
+      if constexpr (PL == 4) {
+        *reinterpret_cast<uint2*>(sdst) = make_uint2(pk[0], pk[1]);
+        *reinterpret_cast<uint2*>(gdst) = make_uint2(pk[0], pk[1]);
+      } else {
+        *reinterpret_cast<uint32_t*>(sdst) = pk[0];
+        *reinterpret_cast<uint32_t*>(gdst) = pk[0];
+      }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    // z_j: column sums of the (bf16) phi values, rows ascending
+    if (threadIdx.x < D) {
+      const int c = threadIdx.x;
+      float z = 0.0f;
+      for (int r = 0; r < 64; ++r) z += bf2f(PK[swz(r, c, D)]);
+      zblk[(size_t(bh) * Nb + jb) * D + c] = z;
+    }
+    // H_chunk += phi(K_j)^T V_j : A = phi(K)^T (m = dim, k = token), B = V
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t a[4];
+      {
+        const int tr = 16 * kk + (lane & 7) + ((lane >> 4) << 3);
+        const int tc = 16 * mt + (((lane >> 3) & 1) << 3);
+        ldsm_x4_t(smem_u32(PK + swz(tr, tc, D)), a[0], a[1], a[2], a[3]);
+      }
+#pragma unroll
+      for (int q = 0; q < NT / 2; ++q) {
+        uint32_t b0, b1, b2, b3;
+        const int tr = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int tc = n0 + 16 * q + ((lane >> 4) << 3);
+        ldsm_x4_t(smem_u32(Vs + swz(tr, tc, D)), b0, b1, b2, b3);
+        mma16816(acc[2 * q], a, b0, b1);
+        mma16816(acc[2 * q + 1], a, b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+  // partial H of this chunk: rows (dims) 16 mt + lane/4 (+8), columns n0 + 8t + 2(lane%4)
+  float* hp = hpart + (size_t(bh) * nchunk + chunk) * D * D;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int r = 16 * mt + (lane >> 2);
+    const int c = n0 + 8 * t + 2 * (lane & 3);
+    *reinterpret_cast<float2*>(hp + size_t(r) * D + c) = make_float2(acc[t][0], acc[t][1]);
+    *reinterpret_cast<float2*>(hp + size_t(r + 8) * D + c) = make_float2(acc[t][2], acc[t][3]);
+  }
+}
+
+cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                           __nv_bfloat16* phik, float* zblk, float* hpart, cudaStream_t s) {
+  dim3 grid(L.nchunk, L.BH);
+  if (L.d == 128)
+    phik_hz_kernel<128><<<grid, 256, 0, s>>>(K, V, phik, zblk, hpart, L.N, L.Npad, L.Nb, L.nchunk);
+  else
+    phik_hz_kernel<64><<<grid, 256, 0, s>>>(K, V, phik, zblk, hpart, L.N, L.Npad, L.Nb, L.nchunk);
+  return cudaGetLastError();
+}
+
+// H_tot = sum over chunks (ascending) -> bf16; Z_tot = sum over blocks (ascending).
+__global__ void __launch_bounds__(256) hz_reduce_kernel(const float* __restrict__ zblk,
+                                                        const float* __restrict__ hpart,
+                                                        __nv_bfloat16* __restrict__ htot16,
+                                                        float* __restrict__ ztot, int Nb, int nchunk,
+                                                        int d) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * 256 + threadIdx.x;
+  const size_t dd = size_t(d) * d;
+  if (e < int(dd)) {
+    const float* src = hpart + size_t(bh) * nchunk * dd + e;
+    float s = 0.0f;
+    for (int c = 0; c < nchunk; ++c) s += src[size_t(c) * dd];
+    htot16[size_t(bh) * dd + e] = __float2bfloat16_rn(s);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < d) {
+    const float* zs = zblk + size_t(bh) * Nb * d + threadIdx.x;
+    float s = 0.0f;
+    for (int j = 0; j < Nb; ++j) s += zs[size_t(j) * d];
+    ztot[size_t(bh) * d + threadIdx.x] = s;
+  }
+}
+
+cudaError_t launch_hz_reduce(const Layout& L, const float* zblk, const float* hpart,
+                             __nv_bfloat16* htot16, float* ztot, cudaStream_t s) {
+  dim3 grid((L.d * L.d + 255) / 256, L.BH);
+  hz_reduce_kernel<<<grid, 256, 0, s>>>(zblk, hpart, htot16, ztot, L.Nb, L.nchunk, L.d);
+  return cudaGetLastError();
+}
+
+}  // namespace sla

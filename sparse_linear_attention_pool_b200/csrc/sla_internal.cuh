@@ -1,0 +1,151 @@
+// Internal declarations shared by the library's translation units: the
+// workspace layout, launcher prototypes and small device helpers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sla.h"
+
+namespace sla {
+
+constexpr int kBlock = SLA_BLOCK;  // bq = bkv = 64 tokens
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Status-word codes written by kernels into the first bytes of the workspace.
+enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1, kDevBadIndex = 2 };
+
+// Tokens per CTA in the phi(K) / h / z pass (16 blocks).
+constexpr int kHzChunk = 1024;
+
+// Derived sizes and the byte offsets of every workspace region.
+struct Layout {
+  int B, H, BH, N, Npad, Nb, d, kc, kn, nchunk;
+  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, htot16, ztot, total;
+};
+
+inline Layout make_layout(const sla_params& p) {
+  Layout L{};
+  L.B = p.B;
+  L.H = p.H;
+  L.BH = p.B * p.H;
+  L.N = p.N;
+  L.Nb = (p.N + kBlock - 1) / kBlock;
+  L.Npad = L.Nb * kBlock;
+  L.d = p.d;
+  L.kc = p.k_crit;
+  L.kn = p.k_neg;
+  L.nchunk = (L.Npad + kHzChunk - 1) / kHzChunk;
+  const size_t BH = size_t(L.BH), Nb = size_t(L.Nb), d = size_t(L.d);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.status = take(256);
+  L.qbar = take(BH * Nb * d * 4);
+  L.kbar = take(BH * Nb * d * 4);
+  L.scores = take(BH * Nb * Nb * 4);
+  L.mc = take(BH * Nb * Nb);
+  L.crit = take(BH * Nb * size_t(L.kc) * 4);
+  L.neg = take(BH * Nb * size_t(L.kn > 0 ? L.kn : 1) * 4);
+  L.phik = take(BH * size_t(L.Npad) * d * 2);
+  L.zblk = take(BH * Nb * d * 4);
+  L.hpart = take(BH * size_t(L.nchunk) * d * d * 4);
+  L.htot16 = take(BH * d * d * 2);
+  L.ztot = take(BH * d * 4);
+  L.total = off;
+  return L;
+}
+
+// ---- launchers (each enqueues on `s`; returns cudaGetLastError()) ----
+cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bfloat16* K,
+                        const __nv_bfloat16* proj_q, const __nv_bfloat16* proj_k, float* qbar,
+                        float* kbar, cudaStream_t s);
+cudaError_t launch_scores(const Layout& L, const float* qbar, const float* kbar, float* scores,
+                          cudaStream_t s);
+cudaError_t launch_classify(const Layout& L, const float* scores, int8_t* mc, int32_t* crit,
+                            int32_t* neg, cudaStream_t s);
+cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                           __nv_bfloat16* phik, float* zblk, float* hpart, cudaStream_t s);
+cudaError_t launch_hz_reduce(const Layout& L, const float* zblk, const float* hpart,
+                             __nv_bfloat16* htot16, float* ztot, cudaStream_t s);
+
+struct AttnArgs {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  __nv_bfloat16* O;
+  const __nv_bfloat16* phik;   // [BH, Npad, d]
+  const int32_t* crit;         // [BH, Nb, kc]
+  const int32_t* neg;          // [BH, Nb, kn]
+  const __nv_bfloat16* htot16; // [BH, d, d]
+  const float* ztot;           // [BH, d]
+  const __nv_bfloat16* w_proj; // [d, d] or null
+  const float* alpha;          // [H] or null
+  int* status;                 // device status word (null: not reported)
+  int H, N, Nb, kc, kn;
+  float scale_log2;            // softmax scale * log2(e)
+};
+enum AttnMode { kModeSLA = 0, kModeSLA2 = 1, kModeDense = 2 };
+cudaError_t launch_attention(const AttnArgs& a, int BH, int d, int mode, cudaStream_t s);
+
+// ---- device helpers ----
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Offset (in elements) of element (row, col) of a bf16 tile with `cols`
+// columns stored with a 16-byte-chunk XOR swizzle (chunk ^= row & 7): makes
+// 8-row ldmatrix reads and 16-byte cp.async writes bank-conflict free.
+__device__ __forceinline__ int swz(int row, int col, int cols) {
+  return row * cols + ((((col >> 3) ^ (row & 7))) << 3) + (col & 7);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  int n = valid ? 16 : 0;  // n = 0 writes 16 zero bytes and reads nothing
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int n>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(n));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two floats -> packed bf16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+}  // namespace sla

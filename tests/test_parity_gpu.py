@@ -1,0 +1,156 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Mask Mc and the critical / negligible lists: bit-exact (both sides rank the
+same float32 pooled scores, ties to the lowest block index). Output O (bf16):
+max-abs <= 2e-2 and relative L2 <= 1e-2 against the unrounded float64 oracle.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+import workloads as W
+from tests.gpu_helpers import (assert_close, device_inputs, errors, oracle_head, oracle_mask_only,
+                               run_library)
+
+pytestmark = pytest.mark.gpu
+
+
+def check_all(sla, inp, o_heads=None, use_w=True, use_router=True, **kw):
+    w = inp.w
+    r = run_library(sla, inp, use_w=use_w, use_router=use_router, **kw)
+    assert r["status"] == 0
+    n_heads = len(inp.heads)
+    o_heads = range(n_heads) if o_heads is None else o_heads
+    flat = lambda a: a.reshape((n_heads,) + a.shape[2:])  # noqa: E731
+    Mc, crit, neg, O = flat(r["Mc"]), flat(r["crit"]), flat(r["neg"]), flat(r["O"])
+    for idx in range(n_heads):
+        if idx in o_heads:
+            ref = oracle_head(inp, idx, use_w=use_w, use_router=use_router)
+        else:
+            ref = oracle_mask_only(inp, idx, use_router=use_router)
+        np.testing.assert_array_equal(Mc[idx], ref["Mc"], err_msg=f"Mc head {inp.heads[idx]}")
+        np.testing.assert_array_equal(crit[idx], ref["crit"])
+        np.testing.assert_array_equal(neg[idx], ref["neg"])
+        if idx in o_heads:
+            assert_close(O[idx][:w.N], ref["O"], what=f"{w.name} head {inp.heads[idx]}")
+    return r
+
+
+def test_tiny_workload_all_heads(cuda_lib):
+    check_all(cuda_lib, W.make_inputs(W.WORKLOADS["sla_b1h2n1024d64"]))
+
+
+EDGE = [
+    # name, B, H, N, d, variant, k_crit, k_neg, use_w, use_router
+    ("ragged_d64_sla", 1, 2, 64 * 5 + 17, 64, "sla", 2, 1, True, True),
+    ("ragged_d128_sla2", 1, 2, 64 * 5 + 17, 128, "sla2", 2, 0, True, True),
+    ("all_critical", 1, 1, 64 * 7, 128, "sla2", 7, 0, True, True),
+    ("empty_marginal_one_row_tail", 1, 2, 64 * 6 + 1, 128, "sla", 3, 4, True, True),
+    ("kn0_d64_sla2", 1, 2, 64 * 6, 64, "sla2", 1, 0, True, True),
+    ("two_blocks", 1, 1, 100, 128, "sla", 1, 0, True, True),
+    ("single_block", 1, 1, 64, 64, "sla2", 1, 0, True, True),
+    ("no_proj_identity", 1, 1, 64 * 9 + 33, 128, "sla", 2, 3, False, True),
+    ("no_router", 1, 1, 64 * 9 + 33, 128, "sla2", 3, 0, True, False),
+    ("batch2_heads3", 2, 3, 64 * 11 + 5, 128, "sla", 3, 2, True, True),
+    ("many_blocks_d64", 1, 1, 64 * 40, 64, "sla", 4, 8, True, True),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
+def test_edge_shapes(cuda_lib, case):
+    name, B, H, N, d, variant, kc, kn, use_w, use_router = case
+    w = W.make_workload(name, B, H, N, d, variant, k_crit=kc, k_neg=kn, cluster_scale=2.0, seed=11)
+    check_all(cuda_lib, W.make_inputs(w), use_w=use_w, use_router=use_router)
+
+
+def test_pad_rows_ignored_and_output_pad_untouched(cuda_lib):
+    w = W.make_workload("pad", 1, 2, 64 * 8 + 23, 128, "sla", k_crit=2, k_neg=2, seed=5)
+    a = run_library(cuda_lib, W.make_inputs(w))
+    b = run_library(cuda_lib, W.make_inputs(w.replace(pad_value=float("nan"))), out_fill=0x7F7F)
+    np.testing.assert_array_equal(a["Mc"], b["Mc"])
+    np.testing.assert_array_equal(a["O"][:, :, :w.N], b["O"][:, :, :w.N])
+    raw = b["O_raw"].view(__import__("torch").int16).cpu().numpy()
+    assert np.all(raw[:, :, w.N:] == 0x7F7F)
+
+
+def test_deterministic_and_workspace_contents_irrelevant(cuda_lib):
+    w = W.make_workload("det", 1, 3, 64 * 20 + 9, 128, "sla", k_crit=3, k_neg=4, seed=6)
+    inp = W.make_inputs(w)
+    dev = device_inputs(inp)
+    a = run_library(cuda_lib, inp, dev=dev)
+    b = run_library(cuda_lib, inp, dev=dev, ws_fill=0xFF)
+    np.testing.assert_array_equal(a["O"][:, :, :w.N], b["O"][:, :, :w.N])  # pad rows are never written
+    np.testing.assert_array_equal(a["Mc"], b["Mc"])
+    np.testing.assert_array_equal(a["crit"], b["crit"])
+
+
+def test_pooled_vectors_match_float32_specification(cuda_lib):
+    w = W.make_workload("pooled", 1, 2, 64 * 9 + 40, 128, "sla2", k_crit=2, k_neg=0, seed=8)
+    inp = W.make_inputs(w)
+    r = run_library(cuda_lib, inp)
+    qb, kb = cuda_lib.get_pooled(r["params"], r["ws"])
+    for idx in range(2):
+        ref = oracle_mask_only(inp, idx)
+        np.testing.assert_array_equal(qb[0, idx].cpu().numpy(), ref["qbar"])
+        np.testing.assert_array_equal(kb[0, idx].cpu().numpy(), ref["kbar"])
+
+
+@pytest.mark.parametrize("N,d", [(64 * 3 + 50, 64), (64 * 10 + 1, 128), (64 * 16, 128)])
+def test_dense_kernel_small(cuda_lib, N, d):
+    import torch
+    from oracle import sla_oracle as O
+
+    w = W.make_workload("dense", 1, 2, N, d, "sla", k_crit=1, k_neg=0, seed=12)
+    inp = W.make_inputs(w)
+    dev = device_inputs(inp)
+    out = torch.zeros_like(dev["q"])
+    cuda_lib.dense_forward(dev["q"], dev["k"], dev["v"], N=N, out=out)
+    torch.cuda.synchronize()
+    from tests.gpu_helpers import from_dev_bf16
+
+    got = from_dev_bf16(out)
+    for h in range(2):
+        q, k, v = (O.bf16_to_f64(x[0, h]) for x in (inp.q, inp.k, inp.v))
+        Mc = np.ones((w.Nb, w.Nb), dtype=np.int8)
+        ref = O.sparse_branch(q, k, v, Mc, N, 1 / math.sqrt(d))
+        assert_close(got[0, h, :N], ref, what=f"dense N={N} d={d}")
+
+
+def test_dense_kernel_full_size_sampled_rows(cuda_lib):
+    import torch
+    from oracle import sla_oracle as O
+    from tests.gpu_helpers import from_dev_bf16
+
+    w = W.WORKLOADS["sla2_b1h12n32768d128_s97"]
+    inp = W.make_inputs(w)
+    dev = device_inputs(inp)
+    out = from_dev_bf16(cuda_lib.dense_forward(dev["q"], dev["k"], dev["v"], N=w.N))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    for h in (0, 7):
+        q, k, v = (O.bf16_to_f64(x[0, h]) for x in (inp.q, inp.k, inp.v))
+        Mc = np.zeros((w.Nb, w.Nb), dtype=np.int8)
+        rows = rng.choice(w.Nb, 3, replace=False)
+        Mc[rows] = 1
+        ref = O.sparse_branch(q, k, v, Mc, w.N, 1 / math.sqrt(w.d))
+        for i in rows:
+            assert_close(out[0, h, i * 64:(i + 1) * 64], ref[i * 64:(i + 1) * 64],
+                         what=f"dense full size head {h} block {i}")
+
+
+@pytest.mark.parametrize("name,o_heads", [
+    ("sla_wan13b_b1h12n32768d128_s95", (0, 11)),
+    ("sla2_b1h12n32768d128_s97", (3, 8)),
+])
+def test_full_size_workloads(cuda_lib, name, o_heads):
+    """Mask bit-exact on every head; O on sampled heads (every row of them)."""
+    check_all(cuda_lib, W.make_inputs(W.WORKLOADS[name]), o_heads=o_heads)
+
+
+def test_wan14b_shape_bf16_path(cuda_lib):
+    """The 14B-720P shape (H=40, N=75600 padded to 75648) through the bf16 path:
+    mask on every head, O on one sampled head."""
+    w = W.WORKLOADS["sla2_q_wan14b_b1h40n75600d128_s97"].replace(precision="bf16")
+    check_all(cuda_lib, W.make_inputs(w), o_heads=(17,))
