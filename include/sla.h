@@ -150,6 +150,33 @@ sla_status sla_read_device_status(const void* workspace, void* stream);
 sla_status sla_dense_forward(const void* Q, const void* K, const void* V, void* O, int B, int H,
                              int N, int d, float softmax_scale, void* stream);
 
+/* Forward pass for callers that cannot allocate device memory (no counterpart
+ * on the pages: it is a deployment aid). Some host programs own all GPU memory
+ * themselves (a plugin inside a server or engine with a fixed memory pool, a
+ * statically planned embedded deployment) or must not call cudaMalloc while
+ * running, since it can synchronise the device. They pass Q, K, V, O and the
+ * parameters exactly as for sla_forward, but no workspace.
+ *
+ * The scratch comes from one static device array of SLA_NOALLOC_WORKSPACE_BYTES
+ * (32 MiB) inside the library, held by every GPU that loads the library until
+ * the process exits. The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *   - Returns SLA_ERR_WORKSPACE, before enqueueing anything, when
+ *     sla_workspace_size(p) exceeds SLA_NOALLOC_WORKSPACE_BYTES.
+ *   - The first call on a device looks up the array's device address for that
+ *     device (cudaGetSymbolAddress, with that device current); make that first
+ *     call before any stream capture begins.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; each call re-initialises what must start at zero. Calls whose
+ *     GPU work overlaps (different streams, different host threads without
+ *     ordering) race on the array and give undefined results: order them on
+ *     one stream or serialise them.
+ *   - The mask, lists and device status of these calls live in the shared
+ *     array and are not readable through sla_get_mask / sla_read_device_status. */
+#define SLA_NOALLOC_WORKSPACE_BYTES (32u << 20)
+sla_status sla_forward_noalloc(const void* Q, const void* K, const void* V, void* O,
+                               const sla_params* p, void* stream);
+
 /* Stage timing, a profiling aid (no counterpart on the pages). Stages of
  * sla_forward, in order: 0 pooling (+ router), 1 pooled scores, 2 classification,
  * 3 phi(K) / z_j / partial H, 4 H_tot / Z_tot reduction, 5 attention (sparse +

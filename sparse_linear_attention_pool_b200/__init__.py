@@ -28,7 +28,8 @@ BLOCK = 64
 # every symbol include/sla.h declares
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate", "sla_workspace_size",
            "sla_forward", "sla_get_mask", "sla_get_pooled", "sla_read_device_status",
-           "sla_dense_forward", "sla_stage_timing", "sla_stage_times")
+           "sla_dense_forward", "sla_stage_timing", "sla_stage_times", "sla_forward_noalloc")
+NOALLOC_WORKSPACE_BYTES = 32 << 20
 NUM_STAGES = 6
 STAGES = ("pool", "scores", "classify", "phik_hz", "hz_reduce", "attention")
 
@@ -75,6 +76,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sla_get_pooled": (i, [P, vp, vp, vp, vp]),
         "sla_read_device_status": (i, [vp, vp]),
         "sla_dense_forward": (i, [vp, vp, vp, vp, i, i, i, i, ctypes.c_float, vp]),
+        "sla_forward_noalloc": (i, [vp, vp, vp, vp, P, vp]),
         "sla_stage_timing": (i, [i]),
         "sla_stage_times": (i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
     }
@@ -216,3 +218,17 @@ def stage_times() -> tuple[dict, int]:
     n = ctypes.c_int(0)
     _check(load().sla_stage_times(ms, ctypes.byref(n)), "sla_stage_times")
     return {name: float(ms[i]) for i, name in enumerate(STAGES)}, n.value
+
+
+def forward_noalloc(q, k, v, *, params: Params, out=None, stream=None):
+    """sla_forward_noalloc: the forward with the library's static scratch array
+    instead of a caller-supplied workspace (for callers that cannot allocate).
+    Calls on one device share that array: do not let their GPU work overlap."""
+    import torch
+
+    if out is None:
+        out = torch.empty_like(q)
+    st = load().sla_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(params),
+                                    _stream(stream))
+    _check(st, "sla_forward_noalloc")
+    return out
