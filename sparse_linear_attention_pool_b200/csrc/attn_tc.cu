@@ -1,0 +1,640 @@
+// Hybrid compute and fusion on the 5th-generation tensor cores (tcgen05).
+//
+// One CTA handles two adjacent 64-row query blocks A and B of one head. Per
+// query block i the method computes ([SLA-sum] = SLA structured summary,
+// aipaper.cc, section 4; [SLA-walk] = SLA walkthrough, intelliparadigm.com):
+//   O^s_i = softmax over the keys of the critical blocks of row i, scale
+//           1/sqrt(d), by online softmax ([SLA-sum] step 3; [SLA-walk] 2.2);
+//   O^l_i = phi(Q_i) H_i / phi(Q_i) Z_i, H_i and Z_i summed over the marginal
+//           blocks ([SLA-sum] formula 3), formed here as
+//           H_i = H_tot - G_i, G_i = sum_{j in E_i} phi(K_j)^T V_j and
+//           Z_i = Z_tot - sum_{j in E_i} z_j, E_i = critical and negligible blocks;
+//   SLA:  O = O^s + O^l W ([SLA-sum] formula 4);
+//   SLA2: O = alpha_h O^s + (1 - alpha_h) O^l (SLA2 article, mcffsbgs.com,
+//         mixing-formula paragraph).
+// Dense mode (the baseline): every key block critical, O = O^s.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax / epilogue: one thread per query row (rows of block A
+//              in TMEM lanes 0-15 of each 32-lane quarter, block B in lanes
+//              16-31: two M=64 accumulators interleaved in the same columns);
+//   warp 4     TMA producer: Q tiles, then per step the K/V tiles of both
+//              blocks (phase 1), then phi(K)/V tiles of the excluded blocks
+//              (phase 2), then W;
+//   warp 5     MMA issuer (one thread) and TMEM owner.
+// Phase 1 per step t: S = Q K_j^T (M=64, N=64) into one of two TMEM S
+// buffers; softmax reads S, writes P (bf16) to shared memory; O += P V_j
+// (M=64, N=d). S(t+1) is issued before PV(t) so the softmax of one step
+// overlaps the tensor core work of the next. O is rescaled in TMEM only when
+// a row maximum grows by more than 2^8 (exponent margin of bf16 P / fp32 O).
+// Phase 2: G += phi(K_j)^T V_j (M=d, N=d) over E_i. Epilogue:
+// H_i = H_tot - G in bf16 -> shared memory, phi(Q_i) in place of Q_i,
+// num = phi(Q_i) H_i on the tensor core, SLA's Y = O^l W likewise.
+//
+// Every wait is bounded (about 2 s); an expired wait sets the device status
+// word to kDevTimeout and makes every later wait of the CTA return at once,
+// so the kernel always terminates.
+#include <string.h>
+
+#include "tc_util.cuh"
+
+namespace sla {
+
+using namespace tc;
+
+struct TcMaps {
+  CUtensorMap q, k, v, phik, w;
+};
+
+template <int D>
+struct TcCfg {
+  static constexpr int kSub = D / 64;          // 64-column sub-tiles of a row
+  static constexpr int kTile = 64 * D * 2;     // bytes of a 64 x D bf16 tile
+  static constexpr int kNS = 2;                // pipeline stages
+  static constexpr int oQA = 0, oQB = kTile;   // Q (later phi(Q)) of blocks A, B
+  static constexpr int oPA = 2 * kTile, oPB = 2 * kTile + 8192;
+  static constexpr int oStage = 2 * kTile + 16384;
+  static constexpr int kStage = 4 * kTile;     // K_A V_A K_B V_B  |  phiK_A V_A phiK_B V_B
+  static constexpr int kMat = D * D * 2;       // D x D bf16
+  static constexpr int oHA = oStage, oHB = oStage + kMat, oW = oStage + 2 * kMat;
+  static constexpr int oOlA = oStage + 3 * kMat, oOlB = oOlA + kTile;
+  static constexpr int kBytes = oStage + kNS * kStage;
+  static_assert(oOlB + kTile <= kBytes, "epilogue tiles must fit in the stage area");
+  // TMEM columns (fp32)
+  static constexpr int cS = 0;                 // S buffers [0,64) and [64,128)
+  static constexpr int cO = 128;               // O: D columns
+  static constexpr int cG = 128 + D;           // G_A (D=128: G_B at cG + 128)
+  static constexpr int cNum = 0;               // num, after the loop
+  static constexpr int cY = cG;                // Y = O^l W, after G is consumed
+  static constexpr uint32_t kTmemCols = D == 128 ? 512 : 256;
+};
+
+enum Bar {
+  bQFull = 0, bKvFull0, bKvFull1, bKvEmpty0, bKvEmpty1, bSFull0, bSFull1, bSFree0, bSFree1,
+  bPFull, bPvDone, bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, kNumBars
+};
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__ TcMaps maps,
+                                                         const AttnArgs a) {
+  using C = TcCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bars[kNumBars];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ float zs[2][D];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y, h = bh % a.H;
+  const int N = a.N, Nb = a.Nb;
+  const int iA = 2 * blockIdx.x;
+  const bool validB = iA + 1 < Nb;
+  const int iB = validB ? iA + 1 : iA;
+  const bool dense = MODE == kModeDense;
+  const int nA = dense ? Nb : a.kc;
+  const bool has_marg = !dense && (a.kc + a.kn < Nb);
+  const int nE = a.kc + a.kn;
+  const bool use_y = MODE == kModeSLA && a.w_proj != nullptr && has_marg;
+  const int32_t* critA = a.crit + (size_t(bh) * Nb + iA) * a.kc;
+  const int32_t* critB = a.crit + (size_t(bh) * Nb + iB) * a.kc;
+  const int kn_stride = a.kn > 0 ? a.kn : 1;
+  const int32_t* negA = a.neg + (size_t(bh) * Nb + iA) * kn_stride;
+  const int32_t* negB = a.neg + (size_t(bh) * Nb + iB) * kn_stride;
+  volatile int* abort_flag = &abort_sh;
+
+  auto checked = [&](int j) {
+    if (j < 0 || j >= Nb) {
+      if (a.status) atomicExch(a.status, kDevBadIndex);
+      j = j < 0 ? 0 : Nb - 1;
+    }
+    return j;
+  };
+  auto crit_block = [&](const int32_t* list, int t) { return dense ? t : checked(list[t]); };
+  auto excl_block = [&](const int32_t* cl, const int32_t* nl, int u) {
+    return checked(u < a.kc ? cl[u] : nl[u - a.kc]);
+  };
+  auto bar = [&](int b) { return smem_u32(&bars[b]); };
+  auto wait = [&](int b, uint32_t parity) { return mbar_wait(bar(b), parity, abort_flag, a.status); };
+  // softmax warps: reconverge after a wait, before warp-collective tcgen05 loads / stores
+  auto wait_w = [&](int b, uint32_t parity) {
+    const bool ok = wait(b, parity);
+    __syncwarp();
+    return ok;
+  };
+  // bounded wait that ignores the abort flag: in-flight copies / MMAs must land before exit
+  int no_abort = 0;
+  auto wait_drain = [&](int b, uint32_t parity) {
+    return mbar_wait(bar(b), parity, reinterpret_cast<volatile int*>(&no_abort), a.status);
+  };
+
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t sQA = sb + C::oQA, sQB = sb + C::oQB, sPA = sb + C::oPA, sPB = sb + C::oPB;
+  const uint32_t sStage = sb + C::oStage;
+  const uint32_t sHA = sb + C::oHA, sHB = sb + C::oHB, sW = sb + C::oW;
+  const uint32_t sOlA = sb + C::oOlA, sOlB = sb + C::oOlB;
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(bar(bQFull), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(bKvFull0 + s), 1);
+      mbar_init(bar(bKvEmpty0 + s), 1);
+      mbar_init(bar(bSFull0 + s), 1);
+      mbar_init(bar(bSFree0 + s), 128);
+    }
+    mbar_init(bar(bPFull), 128);
+    mbar_init(bar(bPvDone), 1);
+    mbar_init(bar(bTailDone), 1);
+    mbar_init(bar(bHiFull), 1);
+    mbar_init(bar(bNumFull), 1);
+    mbar_init(bar(bWFull), 1);
+    mbar_init(bar(bOlFull), 1);
+    mbar_init(bar(bYFull), 1);
+    mbar_init(bar(bDrain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) tmem_alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tmem_base_sh;
+
+  if (warp == 4) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      prefetch_tmap(&maps.q);
+      prefetch_tmap(&maps.k);
+      prefetch_tmap(&maps.v);
+      mbar_expect_tx(bar(bQFull), 2 * C::kTile);
+      for (int s = 0; s < C::kSub; ++s) {
+        tma_load_3d(sQA + s * 8192, &maps.q, bar(bQFull), s * 64, iA * 64, bh);
+        tma_load_3d(sQB + s * 8192, &maps.q, bar(bQFull), s * 64, iB * 64, bh);
+      }
+      for (int t = 0; t < nA; ++t) {
+        const int st = t % C::kNS;
+        wait(bKvEmpty0 + st, ((t / C::kNS) & 1) ^ 1);
+        const int jA = crit_block(critA, t), jB = crit_block(critB, t);
+        const uint32_t base = sStage + st * C::kStage;
+        mbar_expect_tx(bar(bKvFull0 + st), 4 * C::kTile);
+        for (int s = 0; s < C::kSub; ++s) {
+          tma_load_3d(base + s * 8192, &maps.k, bar(bKvFull0 + st), s * 64, jA * 64, bh);
+          tma_load_3d(base + C::kTile + s * 8192, &maps.v, bar(bKvFull0 + st), s * 64, jA * 64, bh);
+          tma_load_3d(base + 2 * C::kTile + s * 8192, &maps.k, bar(bKvFull0 + st), s * 64, jB * 64, bh);
+          tma_load_3d(base + 3 * C::kTile + s * 8192, &maps.v, bar(bKvFull0 + st), s * 64, jB * 64, bh);
+        }
+      }
+      if (has_marg) {
+        for (int u = 0; u < nE; ++u) {
+          const int T = nA + u, st = T % C::kNS;
+          wait(bKvEmpty0 + st, ((T / C::kNS) & 1) ^ 1);
+          const int jA = excl_block(critA, negA, u), jB = excl_block(critB, negB, u);
+          const uint32_t base = sStage + st * C::kStage;
+          mbar_expect_tx(bar(bKvFull0 + st), 4 * C::kTile);
+          for (int s = 0; s < C::kSub; ++s) {
+            tma_load_3d(base + s * 8192, &maps.phik, bar(bKvFull0 + st), s * 64, jA * 64, bh);
+            tma_load_3d(base + C::kTile + s * 8192, &maps.v, bar(bKvFull0 + st), s * 64, jA * 64, bh);
+            tma_load_3d(base + 2 * C::kTile + s * 8192, &maps.phik, bar(bKvFull0 + st), s * 64, jB * 64, bh);
+            tma_load_3d(base + 3 * C::kTile + s * 8192, &maps.v, bar(bKvFull0 + st), s * 64, jB * 64, bh);
+          }
+        }
+      }
+      if (use_y) {  // W reuses the stage area once every loop MMA has completed
+        wait(bTailDone, 0);
+        mbar_expect_tx(bar(bWFull), C::kMat);
+        for (int s = 0; s < C::kSub; ++s) tma_load_2d(sW + s * (D * 128), &maps.w, bar(bWFull), s * 64, 0);
+        wait_drain(bWFull, 0);  // this thread leaves only after its copies have landed
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(64, 64, 0, 0);
+      constexpr uint32_t idPV = idesc_bf16(64, D, 0, 1);
+      constexpr uint32_t idG = idesc_bf16(D, D, 1, 1);
+      constexpr uint32_t idN = idesc_bf16(64, D, 0, 1);
+      constexpr uint32_t laneB = 16u << 16;  // block B's M=64 accumulators start at lane 16
+      wait(bQFull, 0);
+      tc_fence_after();
+      auto issue_pv = [&](int tp) {
+        const int st = tp % C::kNS;
+        wait(bPFull, tp & 1);
+        tc_fence_after();
+        const uint32_t base = sStage + st * C::kStage;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = (tp > 0 || k > 0) ? 1u : 0u;
+          mma_bf16(tb + C::cO, sdesc(sPA + k * 32, 16, 1024),
+                   sdesc(base + C::kTile + k * 2048, 8192, 1024), idPV, acc);
+          mma_bf16(tb + laneB + C::cO, sdesc(sPB + k * 32, 16, 1024),
+                   sdesc(base + 3 * C::kTile + k * 2048, 8192, 1024), idPV, acc);
+        }
+        mma_commit(bar(bPvDone));
+        mma_commit(bar(bKvEmpty0 + st));
+      };
+      for (int t = 0; t < nA; ++t) {
+        const int st = t % C::kNS, b = t & 1;
+        wait(bKvFull0 + st, (t / C::kNS) & 1);
+        wait(bSFree0 + b, ((t >> 1) & 1) ^ 1);
+        tc_fence_after();
+        const uint32_t base = sStage + st * C::kStage;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_bf16(tb + C::cS + b * 64, sdesc(sQA + off, 16, 1024), sdesc(base + off, 16, 1024), idS,
+                   k > 0);
+          mma_bf16(tb + laneB + C::cS + b * 64, sdesc(sQB + off, 16, 1024),
+                   sdesc(base + 2 * C::kTile + off, 16, 1024), idS, k > 0);
+        }
+        mma_commit(bar(bSFull0 + b));
+        if (t > 0) issue_pv(t - 1);
+      }
+      if (nA > 0) issue_pv(nA - 1);
+      if (has_marg) {
+        const uint32_t gA = tb + C::cG;
+        const uint32_t gB = D == 128 ? tb + C::cG + 128 : tb + laneB + C::cG;
+        for (int u = 0; u < nE; ++u) {
+          const int T = nA + u, st = T % C::kNS;
+          wait(bKvFull0 + st, (T / C::kNS) & 1);
+          tc_fence_after();
+          const uint32_t base = sStage + st * C::kStage;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t acc = (u > 0 || k > 0) ? 1u : 0u;
+            mma_bf16(gA, sdesc(base + k * 2048, 8192, 1024), sdesc(base + C::kTile + k * 2048, 8192, 1024),
+                     idG, acc);
+            mma_bf16(gB, sdesc(base + 2 * C::kTile + k * 2048, 8192, 1024),
+                     sdesc(base + 3 * C::kTile + k * 2048, 8192, 1024), idG, acc);
+          }
+          mma_commit(bar(bKvEmpty0 + st));
+        }
+      }
+      mma_commit(bar(bTailDone));
+      if (has_marg) {
+        wait(bHiFull, 0);
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_bf16(tb + C::cNum, sdesc(sQA + off, 16, 1024), sdesc(sHA + k * 2048, D * 128, 1024), idN,
+                   k > 0);
+          mma_bf16(tb + laneB + C::cNum, sdesc(sQB + off, 16, 1024), sdesc(sHB + k * 2048, D * 128, 1024),
+                   idN, k > 0);
+        }
+        mma_commit(bar(bNumFull));
+      }
+      if (use_y) {
+        wait(bWFull, 0);
+        wait(bOlFull, 0);
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+          mma_bf16(tb + C::cY, sdesc(sOlA + off, 16, 1024), sdesc(sW + k * 2048, D * 128, 1024), idN, k > 0);
+          mma_bf16(tb + laneB + C::cY, sdesc(sOlB + off, 16, 1024), sdesc(sW + k * 2048, D * 128, 1024),
+                   idN, k > 0);
+        }
+        mma_commit(bar(bYFull));
+      }
+      // every MMA of this thread has completed before TMEM is released
+      mma_commit(bar(bDrain));
+      wait_drain(bDrain, 0);
+    }
+  } else {
+    // --------------------------- softmax / epilogue ---------------------------
+    const int tid = threadIdx.x;  // 0..127
+    const bool isB = lane >= 16;
+    const int r = 16 * warp + (lane & 15);  // row inside the query block
+    const int blk = isB ? iB : iA;
+    const int grow = blk * 64 + r;          // row inside the head
+    const bool store_row = grow < N && (!isB || validB);
+    const uint32_t tq = tb + (uint32_t(32 * warp) << 16);  // this warp's TMEM lane quarter
+    unsigned char* Prow = smem + (isB ? C::oPB : C::oPA) + r * 128;
+    const int32_t* mycrit = isB ? critB : critA;
+    const float sl2 = a.scale_log2;
+    float m = -INFINITY, l = 0.0f;
+    int pv_seen = -1;  // last step whose PV completion this thread has observed
+
+    for (int t = 0; t < nA; ++t) {
+      const int b = t & 1;
+      wait_w(bSFull0 + b, (t >> 1) & 1);
+      tc_fence_after();
+      float s[64];
+      {
+        float lo[32], hi[32];
+        tmem_ld32(tq + C::cS + b * 64, lo);
+        tmem_ld32(tq + C::cS + b * 64 + 32, hi);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = lo[i];
+          s[32 + i] = hi[i];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(bSFree0 + b));
+      const int j = crit_block(mycrit, t);
+      if (j * 64 + 64 > N) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (j * 64 + i >= N) s[i] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
+      mx *= sl2;
+      if (t == 0) {
+        m = mx;
+      } else if (__any_sync(0xffffffffu, mx > m + 8.0f)) {
+        // some row of this warp grew by more than 2^8: rescale the warp's O rows in TMEM
+        wait_w(bPvDone, (t - 1) & 1);
+        pv_seen = t - 1;
+        tc_fence_after();
+        const float mnew = fmaxf(m, mx);
+        const float corr = ex2(m - mnew);
+        l *= corr;
+        m = mnew;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(tq + C::cO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= corr;
+          tmem_st32(tq + C::cO + c * 32, o);
+        }
+        tmem_wait_st();
+      }
+      uint32_t pk[32];
+      float sum = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = ex2(fmaf(s[2 * i], sl2, -m));
+        const float p1 = ex2(fmaf(s[2 * i + 1], sl2, -m));
+        sum += p0 + p1;
+        pk[i] = pack_bf16(p0, p1);
+      }
+      l += sum;
+      if (t > 0 && pv_seen != t - 1) {  // P buffer is free once PV(t-1) has completed
+        wait(bPvDone, (t - 1) & 1);
+        pv_seen = t - 1;
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(Prow + (uint32_t(c ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(bPFull));
+    }
+    if (nA > 0 && pv_seen != nA - 1) wait_w(bPvDone, (nA - 1) & 1);
+    tc_fence_after();
+    const float inv_l = 1.0f / l;
+
+    float den = 1.0f;
+    if (has_marg) {
+      // Z_i = Z_tot - sum over the excluded blocks of z_j, for blocks A and B
+      const float* zt = a.ztot + size_t(bh) * D;
+      const float* zb = a.zblk + size_t(bh) * Nb * D;
+      for (int e = tid; e < 2 * D; e += 128) {
+        const int X = e / D, c = e % D;
+        const int32_t* cl = X ? critB : critA;
+        const int32_t* nl = X ? negB : negA;
+        float z = zt[c];
+        for (int u = 0; u < nE; ++u) z -= zb[size_t(excl_block(cl, nl, u)) * D + c];
+        zs[X][c] = z;
+      }
+      // phi(Q) of this row, in place of Q (K-major swizzled tile); three passes
+      // over shared memory (max, sum, write) keep the row out of registers
+      unsigned char* Qrow = smem + (isB ? C::oQB : C::oQA);
+      auto qchunk = [&](int c) -> uint4* {
+        return reinterpret_cast<uint4*>(Qrow + (c >> 3) * 8192 + sw128_chunk(r, c & 7));
+      };
+      float qm = -INFINITY;
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 raw = *qchunk(c);
+        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qm = fmaxf(qm, fmaxf(bf16_lo(wv[e]), bf16_hi(wv[e])));
+      }
+      float qs = 0.0f;
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 raw = *qchunk(c);
+        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qs += expf(bf16_lo(wv[e]) - qm) + expf(bf16_hi(wv[e]) - qm);
+      }
+      const float qinv = 1.0f / qs;
+      named_bar(1, 128);  // zs complete
+      den = 0.0f;
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 raw = *qchunk(c);
+        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          pk[e] = pack_bf16(expf(bf16_lo(wv[e]) - qm) * qinv, expf(bf16_hi(wv[e]) - qm) * qinv);
+          den += bf16_lo(pk[e]) * zs[isB][8 * c + 2 * e] + bf16_hi(pk[e]) * zs[isB][8 * c + 2 * e + 1];
+        }
+        *qchunk(c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      // H_i = H_tot - G_i -> bf16, MN-major tile [D rows c][D cols e]
+      wait_w(bTailDone, 0);
+      tc_fence_after();
+      const float* ht = a.htot32 + size_t(bh) * D * D;
+      if (D == 128) {
+#pragma unroll 1
+        for (int X = 0; X < 2; ++X) {
+          const int c = tid;  // TMEM lane = row c of G (M = 128)
+          const uint32_t tg = tq + C::cG + X * 128;
+          unsigned char* Hrow = smem + (X ? C::oHB : C::oHA);
+#pragma unroll 1
+          for (int ch = 0; ch < D / 32; ++ch) {
+            float g[32];
+            tmem_ld32(tg + ch * 32, g);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              const int e0 = ch * 32 + q8 * 8;
+              const float4 h0 = *reinterpret_cast<const float4*>(ht + size_t(c) * D + e0);
+              const float4 h1 = *reinterpret_cast<const float4*>(ht + size_t(c) * D + e0 + 4);
+              const uint4 v = make_uint4(pack_bf16(h0.x - g[q8 * 8 + 0], h0.y - g[q8 * 8 + 1]),
+                                         pack_bf16(h0.z - g[q8 * 8 + 2], h0.w - g[q8 * 8 + 3]),
+                                         pack_bf16(h1.x - g[q8 * 8 + 4], h1.y - g[q8 * 8 + 5]),
+                                         pack_bf16(h1.z - g[q8 * 8 + 6], h1.w - g[q8 * 8 + 7]));
+              *reinterpret_cast<uint4*>(Hrow + (e0 >> 6) * (D * 128) + sw128_chunk(c, (e0 & 63) >> 3)) = v;
+            }
+          }
+        }
+      } else {
+        const int c = r;  // M = 64 layout: block A rows in lanes 0-15, block B in 16-31
+        unsigned char* Hrow = smem + (isB ? C::oHB : C::oHA);
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          float g[32];
+          tmem_ld32(tq + C::cG + ch * 32, g);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const int e0 = ch * 32 + q8 * 8;
+            const float4 h0 = *reinterpret_cast<const float4*>(ht + size_t(c) * D + e0);
+            const float4 h1 = *reinterpret_cast<const float4*>(ht + size_t(c) * D + e0 + 4);
+            const uint4 v = make_uint4(pack_bf16(h0.x - g[q8 * 8 + 0], h0.y - g[q8 * 8 + 1]),
+                                       pack_bf16(h0.z - g[q8 * 8 + 2], h0.w - g[q8 * 8 + 3]),
+                                       pack_bf16(h1.x - g[q8 * 8 + 4], h1.y - g[q8 * 8 + 5]),
+                                       pack_bf16(h1.z - g[q8 * 8 + 6], h1.w - g[q8 * 8 + 7]));
+            *reinterpret_cast<uint4*>(Hrow + (e0 >> 6) * (D * 128) + sw128_chunk(c, (e0 & 63) >> 3)) = v;
+          }
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      named_bar(1, 128);
+      if (tid == 0) mbar_arrive(bar(bHiFull));
+      wait_w(bNumFull, 0);
+      tc_fence_after();
+    }
+
+    const float alpha = MODE == kModeSLA2 ? a.alpha[h] : 0.0f;
+    const float inv_den = 1.0f / den;
+    __nv_bfloat16* orow = a.O + (size_t(bh) * (size_t(Nb) * 64) + grow) * D;
+    if (use_y) {
+      // O^l (bf16) -> K-major tile, then Y = O^l W on the tensor core
+      unsigned char* Olrow = smem + (isB ? C::oOlB : C::oOlA);
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float nm[32];
+        tmem_ld32(tq + C::cNum + ch * 32, nm);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const int e0 = ch * 32 + q8 * 8;
+          const uint4 v = make_uint4(pack_bf16(nm[q8 * 8 + 0] * inv_den, nm[q8 * 8 + 1] * inv_den),
+                                     pack_bf16(nm[q8 * 8 + 2] * inv_den, nm[q8 * 8 + 3] * inv_den),
+                                     pack_bf16(nm[q8 * 8 + 4] * inv_den, nm[q8 * 8 + 5] * inv_den),
+                                     pack_bf16(nm[q8 * 8 + 6] * inv_den, nm[q8 * 8 + 7] * inv_den));
+          *reinterpret_cast<uint4*>(Olrow + (e0 >> 6) * 8192 + sw128_chunk(r, (e0 & 63) >> 3)) = v;
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      named_bar(1, 128);
+      if (tid == 0) mbar_arrive(bar(bOlFull));
+      wait_w(bYFull, 0);
+      tc_fence_after();
+    }
+#pragma unroll 1
+    for (int ch = 0; ch < D / 32; ++ch) {
+      float o[32], x[32];
+      tmem_ld32(tq + C::cO + ch * 32, o);
+      if (use_y) tmem_ld32(tq + C::cY + ch * 32, x);
+      else if (has_marg) tmem_ld32(tq + C::cNum + ch * 32, x);
+      tmem_wait_ld();
+      float out[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float os = o[i] * inv_l;
+        const float ol = use_y ? x[i] : (has_marg ? x[i] * inv_den : 0.0f);
+        out[i] = MODE == kModeSLA2 ? alpha * os + (1.0f - alpha) * ol : os + ol;
+      }
+      if (store_row) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+          dst[q8] = make_uint4(pack_bf16(out[8 * q8], out[8 * q8 + 1]), pack_bf16(out[8 * q8 + 2], out[8 * q8 + 3]),
+                               pack_bf16(out[8 * q8 + 4], out[8 * q8 + 5]), pack_bf16(out[8 * q8 + 6], out[8 * q8 + 7]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tb, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [BH][rows_alloc][D] bf16 viewed as 3D (D, rows, BH); rows >= rows_valid read as zero.
+bool map_rows(CUtensorMap* m, const void* base, int D, int rows_valid, int rows_alloc, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(rows_valid), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(rows_alloc) * D * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [D][D] bf16 (row = input dim), boxes of 64 columns x D rows.
+bool map_square(CUtensorMap* m, const void* base, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(D)};
+  cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+  cuuint32_t box[2] = {64, cuuint32_t(D)};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int MODE>
+cudaError_t launch_tc(const TcMaps& maps, const AttnArgs& a, int BH, cudaStream_t s) {
+  const int bytes = TcCfg<D>::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       bytes);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<D, MODE><<<dim3((a.Nb + 1) / 2, BH), 192, bytes, s>>>(maps, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnArgs& a, int BH, int d, int mode, cudaStream_t s) {
+  TcMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const int Npad = a.Nb * kBlock;
+  bool ok = map_rows(&maps.q, a.Q, d, a.N, Npad, BH) && map_rows(&maps.k, a.K, d, a.N, Npad, BH) &&
+            map_rows(&maps.v, a.V, d, a.N, Npad, BH);
+  if (ok && a.phik) ok = map_rows(&maps.phik, a.phik, d, Npad, Npad, BH);
+  if (ok && a.w_proj) ok = map_square(&maps.w, a.w_proj, d);
+  if (!ok) return cudaErrorInvalidValue;
+  if (d == 128) {
+    if (mode == kModeSLA) return launch_tc<128, kModeSLA>(maps, a, BH, s);
+    if (mode == kModeSLA2) return launch_tc<128, kModeSLA2>(maps, a, BH, s);
+    return launch_tc<128, kModeDense>(maps, a, BH, s);
+  }
+  if (mode == kModeSLA) return launch_tc<64, kModeSLA>(maps, a, BH, s);
+  if (mode == kModeSLA2) return launch_tc<64, kModeSLA2>(maps, a, BH, s);
+  return launch_tc<64, kModeDense>(maps, a, BH, s);
+}
+
+}  // namespace sla

@@ -151,10 +151,10 @@ cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_b
   return cudaGetLastError();
 }
 
-// H_tot = sum over chunks (ascending) -> bf16; Z_tot = sum over blocks (ascending).
+// H_tot = sum over chunks (ascending); Z_tot = sum over blocks (ascending).
 __global__ void __launch_bounds__(256) hz_reduce_kernel(const float* __restrict__ zblk,
                                                         const float* __restrict__ hpart,
-                                                        __nv_bfloat16* __restrict__ htot16,
+                                                        float* __restrict__ htot32,
                                                         float* __restrict__ ztot, int Nb, int nchunk,
                                                         int d) {
   const int bh = blockIdx.y;
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(256) hz_reduce_kernel(const float* __restrict_
     const float* src = hpart + size_t(bh) * nchunk * dd + e;
     float s = 0.0f;
     for (int c = 0; c < nchunk; ++c) s += src[size_t(c) * dd];
-    htot16[size_t(bh) * dd + e] = __float2bfloat16_rn(s);
+    htot32[size_t(bh) * dd + e] = s;
   }
   if (blockIdx.x == 0 && threadIdx.x < d) {
     const float* zs = zblk + size_t(bh) * Nb * d + threadIdx.x;
@@ -174,10 +174,10 @@ __global__ void __launch_bounds__(256) hz_reduce_kernel(const float* __restrict_
   }
 }
 
-cudaError_t launch_hz_reduce(const Layout& L, const float* zblk, const float* hpart,
-                             __nv_bfloat16* htot16, float* ztot, cudaStream_t s) {
+cudaError_t launch_hz_reduce(const Layout& L, const float* zblk, const float* hpart, float* htot32,
+                             float* ztot, cudaStream_t s) {
   dim3 grid((L.d * L.d + 255) / 256, L.BH);
-  hz_reduce_kernel<<<grid, 256, 0, s>>>(zblk, hpart, htot16, ztot, L.Nb, L.nchunk, L.d);
+  hz_reduce_kernel<<<grid, 256, 0, s>>>(zblk, hpart, htot32, ztot, L.Nb, L.nchunk, L.d);
   return cudaGetLastError();
 }
 

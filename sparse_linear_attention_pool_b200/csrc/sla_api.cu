@@ -97,7 +97,7 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   __nv_bfloat16* phik = reinterpret_cast<__nv_bfloat16*>(ws + L.phik);
   float* zblk = reinterpret_cast<float*>(ws + L.zblk);
   float* hpart = reinterpret_cast<float*>(ws + L.hpart);
-  __nv_bfloat16* htot16 = reinterpret_cast<__nv_bfloat16*>(ws + L.htot16);
+  float* htot32 = reinterpret_cast<float*>(ws + L.htot32);
   float* ztot = reinterpret_cast<float*>(ws + L.ztot);
   const bool sla2 = p->variant == SLA_VARIANT_SLA2;
 
@@ -117,7 +117,7 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   mark(3);
   if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, s);
   mark(4);
-  if (e == cudaSuccess) e = launch_hz_reduce(L, zblk, hpart, htot16, ztot, s);
+  if (e == cudaSuccess) e = launch_hz_reduce(L, zblk, hpart, htot32, ztot, s);
   mark(5);
   if (e == cudaSuccess) {
     AttnArgs a{};
@@ -128,8 +128,9 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
     a.phik = phik;
     a.crit = crit;
     a.neg = neg;
-    a.htot16 = htot16;
+    a.htot32 = htot32;
     a.ztot = ztot;
+    a.zblk = zblk;
     a.w_proj = sla2 ? nullptr : bf(p->w_proj);
     a.alpha = sla2 ? p->alpha : nullptr;
     a.status = reinterpret_cast<int*>(ws + L.status);

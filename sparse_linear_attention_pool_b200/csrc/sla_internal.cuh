@@ -23,7 +23,7 @@ constexpr int kHzChunk = 1024;
 // Derived sizes and the byte offsets of every workspace region.
 struct Layout {
   int B, H, BH, N, Npad, Nb, d, kc, kn, nchunk;
-  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, htot16, ztot, total;
+  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, htot32, ztot, total;
 };
 
 inline Layout make_layout(const sla_params& p) {
@@ -55,7 +55,7 @@ inline Layout make_layout(const sla_params& p) {
   L.phik = take(BH * size_t(L.Npad) * d * 2);
   L.zblk = take(BH * Nb * d * 4);
   L.hpart = take(BH * size_t(L.nchunk) * d * d * 4);
-  L.htot16 = take(BH * d * d * 2);
+  L.htot32 = take(BH * d * d * 4);
   L.ztot = take(BH * d * 4);
   L.total = off;
   return L;
@@ -71,8 +71,8 @@ cudaError_t launch_classify(const Layout& L, const float* scores, int8_t* mc, in
                             int32_t* neg, cudaStream_t s);
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                            __nv_bfloat16* phik, float* zblk, float* hpart, cudaStream_t s);
-cudaError_t launch_hz_reduce(const Layout& L, const float* zblk, const float* hpart,
-                             __nv_bfloat16* htot16, float* ztot, cudaStream_t s);
+cudaError_t launch_hz_reduce(const Layout& L, const float* zblk, const float* hpart, float* htot32,
+                             float* ztot, cudaStream_t s);
 
 struct AttnArgs {
   const __nv_bfloat16* Q;
@@ -82,8 +82,9 @@ struct AttnArgs {
   const __nv_bfloat16* phik;   // [BH, Npad, d]
   const int32_t* crit;         // [BH, Nb, kc]
   const int32_t* neg;          // [BH, Nb, kn]
-  const __nv_bfloat16* htot16; // [BH, d, d]
-  const float* ztot;           // [BH, d]
+  const float* htot32;         // [BH, d, d]  H_tot = sum_j phi(K_j)^T V_j
+  const float* ztot;           // [BH, d]     Z_tot = sum_j z_j
+  const float* zblk;           // [BH, Nb, d] z_j
   const __nv_bfloat16* w_proj; // [d, d] or null
   const float* alpha;          // [H] or null
   int* status;                 // device status word (null: not reported)
