@@ -12,24 +12,28 @@
 //   SLA:  O = O^s + O^l W ([SLA-sum] formula 4);
 //   SLA2: O = alpha_h O^s + (1 - alpha_h) O^l (SLA2 article, mcffsbgs.com,
 //         mixing-formula paragraph).
-// Dense mode (the baseline): every key block critical, O = O^s.
+// Dense mode (the baseline): every key block critical, O = O^s; both query
+// blocks then read the same K/V tile at every step, which is loaded once.
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax / epilogue: one thread per query row (rows of block A
 //              in TMEM lanes 0-15 of each 32-lane quarter, block B in lanes
 //              16-31: two M=64 accumulators interleaved in the same columns);
-//   warp 4     TMA producer: Q tiles, then per step the K/V tiles of both
-//              blocks (phase 1), then phi(K)/V tiles of the excluded blocks
-//              (phase 2), then W;
+//   warp 4     TMA producer: Q tiles, then per step the K and V tiles of both
+//              blocks (phase 1), then the phi(K) / V tiles of the excluded
+//              blocks (phase 2), then W;
 //   warp 5     MMA issuer (one thread) and TMEM owner.
+// K tiles and V tiles travel in separate rings: a K slot is released as soon
+// as the S products that read it complete, a V slot after its PV product.
 // Phase 1 per step t: S = Q K_j^T (M=64, N=64) into one of two TMEM S
-// buffers; softmax reads S, writes P (bf16) to shared memory; O += P V_j
-// (M=64, N=d). S(t+1) is issued before PV(t) so the softmax of one step
-// overlaps the tensor core work of the next. O is rescaled in TMEM only when
-// a row maximum grows by more than 2^8 (exponent margin of bf16 P / fp32 O).
-// Phase 2: G += phi(K_j)^T V_j (M=d, N=d) over E_i. Epilogue:
-// H_i = H_tot - G in bf16 -> shared memory, phi(Q_i) in place of Q_i,
-// num = phi(Q_i) H_i on the tensor core, SLA's Y = O^l W likewise.
+// buffers; the softmax reads S and writes P (bf16) into one of two shared
+// buffers; O += P V_j (M=64, N=d). S(t+1) is issued before PV(t), so the
+// softmax of one step overlaps the tensor-core work of the next. O is
+// rescaled in TMEM only when a row maximum grows by more than 2^8 (the
+// exponent headroom of bf16 P and fp32 O). Phase 2: G += phi(K_j)^T V_j (M=d,
+// N=d) over E_i. Epilogue: H_i = H_tot - G in bf16 -> shared memory, phi(Q_i)
+// in place of Q_i, num = phi(Q_i) H_i on the tensor core, SLA's Y = O^l W
+// likewise.
 //
 // Every wait is bounded (about 2 s); an expired wait sets the device status
 // word to kDevTimeout and makes every later wait of the CTA return at once,
@@ -50,16 +54,19 @@ template <int D>
 struct TcCfg {
   static constexpr int kSub = D / 64;          // 64-column sub-tiles of a row
   static constexpr int kTile = 64 * D * 2;     // bytes of a 64 x D bf16 tile
-  static constexpr int kNS = 2;                // pipeline stages
+  static constexpr int kNK = D == 128 ? 3 : 2; // K-ring slots (K_A, K_B | phiK_A, phiK_B)
+  static constexpr int kNV = 2;                // V-ring slots (V_A, V_B)
+  static constexpr int kPair = 2 * kTile;      // bytes of one ring slot
   static constexpr int oQA = 0, oQB = kTile;   // Q (later phi(Q)) of blocks A, B
-  static constexpr int oPA = 2 * kTile, oPB = 2 * kTile + 8192;
-  static constexpr int oStage = 2 * kTile + 16384;
-  static constexpr int kStage = 4 * kTile;     // K_A V_A K_B V_B  |  phiK_A V_A phiK_B V_B
+  static constexpr int oP = 2 * kTile;         // P buffers: [2 steps][A, B] x 8 KB
+  static constexpr int oK = oP + 4 * 8192;
+  static constexpr int oV = oK + kNK * kPair;
+  static constexpr int kBytes = oV + kNV * kPair;
+  // epilogue tiles reuse the rings once every loop product has completed
   static constexpr int kMat = D * D * 2;       // D x D bf16
-  static constexpr int oHA = oStage, oHB = oStage + kMat, oW = oStage + 2 * kMat;
-  static constexpr int oOlA = oStage + 3 * kMat, oOlB = oOlA + kTile;
-  static constexpr int kBytes = oStage + kNS * kStage;
-  static_assert(oOlB + kTile <= kBytes, "epilogue tiles must fit in the stage area");
+  static constexpr int oHA = oK, oHB = oK + kMat, oW = oK + 2 * kMat;
+  static constexpr int oOlA = oK + 3 * kMat, oOlB = oOlA + kTile;
+  static_assert(oOlB + kTile <= kBytes, "epilogue tiles must fit in the rings");
   // TMEM columns (fp32)
   static constexpr int cS = 0;                 // S buffers [0,64) and [64,128)
   static constexpr int cO = 128;               // O: D columns
@@ -70,8 +77,11 @@ struct TcCfg {
 };
 
 enum Bar {
-  bQFull = 0, bKvFull0, bKvFull1, bKvEmpty0, bKvEmpty1, bSFull0, bSFull1, bSFree0, bSFree1,
-  bPFull, bPvDone, bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, kNumBars
+  bQFull = 0,
+  bKFull0, bKFull1, bKFull2, bKEmpty0, bKEmpty1, bKEmpty2,
+  bVFull0, bVFull1, bVEmpty0, bVEmpty1,
+  bSFull0, bSFull1, bSFree0, bSFree1, bPFull0, bPFull1, bPvDone0, bPvDone1,
+  bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, kNumBars
 };
 
 template <int D, int MODE>
@@ -92,10 +102,11 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   const int iA = 2 * blockIdx.x;
   const bool validB = iA + 1 < Nb;
   const int iB = validB ? iA + 1 : iA;
-  const bool dense = MODE == kModeDense;
+  constexpr bool dense = MODE == kModeDense;
   const int nA = dense ? Nb : a.kc;
   const bool has_marg = !dense && (a.kc + a.kn < Nb);
   const int nE = a.kc + a.kn;
+  const int nTot = nA + (has_marg ? nE : 0);  // ring steps: phase 1 then phase 2
   const bool use_y = MODE == kModeSLA && a.w_proj != nullptr && has_marg;
   const int32_t* critA = a.crit + (size_t(bh) * Nb + iA) * a.kc;
   const int32_t* critB = a.crit + (size_t(bh) * Nb + iB) * a.kc;
@@ -111,13 +122,18 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     }
     return j;
   };
-  auto crit_block = [&](const int32_t* list, int t) { return dense ? t : checked(list[t]); };
-  auto excl_block = [&](const int32_t* cl, const int32_t* nl, int u) {
+  // key block of ring step T for block A (X = 0) or B (X = 1)
+  auto step_block = [&](int X, int T) {
+    if (dense) return T;
+    const int32_t* cl = X ? critB : critA;
+    const int32_t* nl = X ? negB : negA;
+    if (T < nA) return checked(cl[T]);
+    const int u = T - nA;
     return checked(u < a.kc ? cl[u] : nl[u - a.kc]);
   };
   auto bar = [&](int b) { return smem_u32(&bars[b]); };
   auto wait = [&](int b, uint32_t parity) { return mbar_wait(bar(b), parity, abort_flag, a.status); };
-  // softmax warps: reconverge after a wait, before warp-collective tcgen05 loads / stores
+  // reconverge the warp after a wait, before warp-collective tcgen05 loads / stores
   auto wait_w = [&](int b, uint32_t parity) {
     const bool ok = wait(b, parity);
     __syncwarp();
@@ -130,22 +146,28 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   };
 
   const uint32_t sb = smem_u32(smem);
-  const uint32_t sQA = sb + C::oQA, sQB = sb + C::oQB, sPA = sb + C::oPA, sPB = sb + C::oPB;
-  const uint32_t sStage = sb + C::oStage;
+  const uint32_t sQA = sb + C::oQA, sQB = sb + C::oQB, sP = sb + C::oP;
+  const uint32_t sK = sb + C::oK, sV = sb + C::oV;
   const uint32_t sHA = sb + C::oHA, sHB = sb + C::oHB, sW = sb + C::oW;
   const uint32_t sOlA = sb + C::oOlA, sOlB = sb + C::oOlB;
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
     mbar_init(bar(bQFull), 1);
+    for (int s = 0; s < C::kNK; ++s) {
+      mbar_init(bar(bKFull0 + s), 1);
+      mbar_init(bar(bKEmpty0 + s), 1);
+    }
+    for (int s = 0; s < C::kNV; ++s) {
+      mbar_init(bar(bVFull0 + s), 1);
+      mbar_init(bar(bVEmpty0 + s), 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(bKvFull0 + s), 1);
-      mbar_init(bar(bKvEmpty0 + s), 1);
       mbar_init(bar(bSFull0 + s), 1);
       mbar_init(bar(bSFree0 + s), 128);
+      mbar_init(bar(bPFull0 + s), 128);
+      mbar_init(bar(bPvDone0 + s), 1);
     }
-    mbar_init(bar(bPFull), 128);
-    mbar_init(bar(bPvDone), 1);
     mbar_init(bar(bTailDone), 1);
     mbar_init(bar(bHiFull), 1);
     mbar_init(bar(bNumFull), 1);
@@ -163,49 +185,72 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 
   if (warp == 4) {
     // ------------------------------ TMA producer ------------------------------
+    // The whole warp walks the steps; lane i prefetches the block indices of
+    // 32 consecutive steps and lane 0 issues the copies.
     if (lane == 0) {
       prefetch_tmap(&maps.q);
       prefetch_tmap(&maps.k);
       prefetch_tmap(&maps.v);
+      if (has_marg) prefetch_tmap(&maps.phik);
       mbar_expect_tx(bar(bQFull), 2 * C::kTile);
       for (int s = 0; s < C::kSub; ++s) {
         tma_load_3d(sQA + s * 8192, &maps.q, bar(bQFull), s * 64, iA * 64, bh);
         tma_load_3d(sQB + s * 8192, &maps.q, bar(bQFull), s * 64, iB * 64, bh);
       }
-      for (int t = 0; t < nA; ++t) {
-        const int st = t % C::kNS;
-        wait(bKvEmpty0 + st, ((t / C::kNS) & 1) ^ 1);
-        const int jA = crit_block(critA, t), jB = crit_block(critB, t);
-        const uint32_t base = sStage + st * C::kStage;
-        mbar_expect_tx(bar(bKvFull0 + st), 4 * C::kTile);
-        for (int s = 0; s < C::kSub; ++s) {
-          tma_load_3d(base + s * 8192, &maps.k, bar(bKvFull0 + st), s * 64, jA * 64, bh);
-          tma_load_3d(base + C::kTile + s * 8192, &maps.v, bar(bKvFull0 + st), s * 64, jA * 64, bh);
-          tma_load_3d(base + 2 * C::kTile + s * 8192, &maps.k, bar(bKvFull0 + st), s * 64, jB * 64, bh);
-          tma_load_3d(base + 3 * C::kTile + s * 8192, &maps.v, bar(bKvFull0 + st), s * 64, jB * 64, bh);
-        }
+    }
+    const int tileBytes = dense ? C::kTile : 2 * C::kTile;  // dense: one shared tile per step
+    constexpr int lag = C::kNK - C::kNV;  // K copies run this many steps ahead of V copies
+    int kA_reg = 0, kB_reg = 0;           // indices of the current 32-step window (K side)
+    int vA_reg = 0, vB_reg = 0;           // indices of the window the V side reads
+    for (int T = 0; T < nTot + lag; ++T) {
+      const int TK = T, TV = T - lag;
+      if ((TK & 31) == 0 && TK < nTot) {
+        const int Ti = TK + lane;
+        kA_reg = Ti < nTot ? step_block(0, Ti) : 0;
+        kB_reg = Ti < nTot ? step_block(1, Ti) : 0;
       }
-      if (has_marg) {
-        for (int u = 0; u < nE; ++u) {
-          const int T = nA + u, st = T % C::kNS;
-          wait(bKvEmpty0 + st, ((T / C::kNS) & 1) ^ 1);
-          const int jA = excl_block(critA, negA, u), jB = excl_block(critB, negB, u);
-          const uint32_t base = sStage + st * C::kStage;
-          mbar_expect_tx(bar(bKvFull0 + st), 4 * C::kTile);
+      if (TV >= 0 && (TV & 31) == 0 && TV < nTot) {
+        const int Ti = TV + lane;
+        vA_reg = Ti < nTot ? step_block(0, Ti) : 0;
+        vB_reg = Ti < nTot ? step_block(1, Ti) : 0;
+      }
+      if (TK < nTot) {
+        const int jA = __shfl_sync(0xffffffffu, kA_reg, TK & 31);
+        const int jB = __shfl_sync(0xffffffffu, kB_reg, TK & 31);
+        const int st = TK % C::kNK;
+        wait(bKEmpty0 + st, ((TK / C::kNK) & 1) ^ 1);
+        if (lane == 0) {
+          const CUtensorMap* km = TK < nA ? &maps.k : &maps.phik;
+          const uint32_t slot = sK + st * C::kPair;
+          mbar_expect_tx(bar(bKFull0 + st), tileBytes);
           for (int s = 0; s < C::kSub; ++s) {
-            tma_load_3d(base + s * 8192, &maps.phik, bar(bKvFull0 + st), s * 64, jA * 64, bh);
-            tma_load_3d(base + C::kTile + s * 8192, &maps.v, bar(bKvFull0 + st), s * 64, jA * 64, bh);
-            tma_load_3d(base + 2 * C::kTile + s * 8192, &maps.phik, bar(bKvFull0 + st), s * 64, jB * 64, bh);
-            tma_load_3d(base + 3 * C::kTile + s * 8192, &maps.v, bar(bKvFull0 + st), s * 64, jB * 64, bh);
+            tma_load_3d(slot + s * 8192, km, bar(bKFull0 + st), s * 64, jA * 64, bh);
+            if (!dense) tma_load_3d(slot + C::kTile + s * 8192, km, bar(bKFull0 + st), s * 64, jB * 64, bh);
           }
         }
+        __syncwarp();
       }
-      if (use_y) {  // W reuses the stage area once every loop MMA has completed
-        wait(bTailDone, 0);
-        mbar_expect_tx(bar(bWFull), C::kMat);
-        for (int s = 0; s < C::kSub; ++s) tma_load_2d(sW + s * (D * 128), &maps.w, bar(bWFull), s * 64, 0);
-        wait_drain(bWFull, 0);  // this thread leaves only after its copies have landed
+      if (TV >= 0 && TV < nTot) {
+        const int jA = __shfl_sync(0xffffffffu, vA_reg, TV & 31);
+        const int jB = __shfl_sync(0xffffffffu, vB_reg, TV & 31);
+        const int st = TV % C::kNV;
+        wait(bVEmpty0 + st, ((TV / C::kNV) & 1) ^ 1);
+        if (lane == 0) {
+          const uint32_t slot = sV + st * C::kPair;
+          mbar_expect_tx(bar(bVFull0 + st), tileBytes);
+          for (int s = 0; s < C::kSub; ++s) {
+            tma_load_3d(slot + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jA * 64, bh);
+            if (!dense) tma_load_3d(slot + C::kTile + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jB * 64, bh);
+          }
+        }
+        __syncwarp();
       }
+    }
+    if (use_y && lane == 0) {  // W reuses the rings once every loop product has completed
+      wait(bTailDone, 0);
+      mbar_expect_tx(bar(bWFull), C::kMat);
+      for (int s = 0; s < C::kSub; ++s) tma_load_2d(sW + s * (D * 128), &maps.w, bar(bWFull), s * 64, 0);
+      wait_drain(bWFull, 0);  // leave only after the copies have landed
     }
   } else if (warp == 5) {
     // ------------------------------ MMA issuer ------------------------------
@@ -215,39 +260,41 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       constexpr uint32_t idG = idesc_bf16(D, D, 1, 1);
       constexpr uint32_t idN = idesc_bf16(64, D, 0, 1);
       constexpr uint32_t laneB = 16u << 16;  // block B's M=64 accumulators start at lane 16
+      const uint32_t tileB = dense ? 0u : uint32_t(C::kTile);  // dense: B reads A's tile
       wait(bQFull, 0);
       tc_fence_after();
       auto issue_pv = [&](int tp) {
-        const int st = tp % C::kNS;
-        wait(bPFull, tp & 1);
+        const int stv = tp % C::kNV, pb = tp & 1;
+        wait(bVFull0 + stv, (tp / C::kNV) & 1);
+        wait(bPFull0 + pb, (tp >> 1) & 1);
         tc_fence_after();
-        const uint32_t base = sStage + st * C::kStage;
+        const uint32_t vslot = sV + stv * C::kPair;
+        const uint32_t pA = sP + pb * 16384, pB = pA + 8192;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint32_t acc = (tp > 0 || k > 0) ? 1u : 0u;
-          mma_bf16(tb + C::cO, sdesc(sPA + k * 32, 16, 1024),
-                   sdesc(base + C::kTile + k * 2048, 8192, 1024), idPV, acc);
-          mma_bf16(tb + laneB + C::cO, sdesc(sPB + k * 32, 16, 1024),
-                   sdesc(base + 3 * C::kTile + k * 2048, 8192, 1024), idPV, acc);
+          mma_bf16(tb + C::cO, sdesc(pA + k * 32, 16, 1024), sdesc(vslot + k * 2048, 8192, 1024), idPV, acc);
+          mma_bf16(tb + laneB + C::cO, sdesc(pB + k * 32, 16, 1024),
+                   sdesc(vslot + tileB + k * 2048, 8192, 1024), idPV, acc);
         }
-        mma_commit(bar(bPvDone));
-        mma_commit(bar(bKvEmpty0 + st));
+        mma_commit(bar(bPvDone0 + pb));
+        mma_commit(bar(bVEmpty0 + stv));
       };
       for (int t = 0; t < nA; ++t) {
-        const int st = t % C::kNS, b = t & 1;
-        wait(bKvFull0 + st, (t / C::kNS) & 1);
+        const int stk = t % C::kNK, b = t & 1;
+        wait(bKFull0 + stk, (t / C::kNK) & 1);
         wait(bSFree0 + b, ((t >> 1) & 1) ^ 1);
         tc_fence_after();
-        const uint32_t base = sStage + st * C::kStage;
+        const uint32_t kslot = sK + stk * C::kPair;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_bf16(tb + C::cS + b * 64, sdesc(sQA + off, 16, 1024), sdesc(base + off, 16, 1024), idS,
-                   k > 0);
+          mma_bf16(tb + C::cS + b * 64, sdesc(sQA + off, 16, 1024), sdesc(kslot + off, 16, 1024), idS, k > 0);
           mma_bf16(tb + laneB + C::cS + b * 64, sdesc(sQB + off, 16, 1024),
-                   sdesc(base + 2 * C::kTile + off, 16, 1024), idS, k > 0);
+                   sdesc(kslot + tileB + off, 16, 1024), idS, k > 0);
         }
         mma_commit(bar(bSFull0 + b));
+        mma_commit(bar(bKEmpty0 + stk));
         if (t > 0) issue_pv(t - 1);
       }
       if (nA > 0) issue_pv(nA - 1);
@@ -255,19 +302,20 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         const uint32_t gA = tb + C::cG;
         const uint32_t gB = D == 128 ? tb + C::cG + 128 : tb + laneB + C::cG;
         for (int u = 0; u < nE; ++u) {
-          const int T = nA + u, st = T % C::kNS;
-          wait(bKvFull0 + st, (T / C::kNS) & 1);
+          const int T = nA + u, stk = T % C::kNK, stv = T % C::kNV;
+          wait(bKFull0 + stk, (T / C::kNK) & 1);
+          wait(bVFull0 + stv, (T / C::kNV) & 1);
           tc_fence_after();
-          const uint32_t base = sStage + st * C::kStage;
+          const uint32_t kslot = sK + stk * C::kPair, vslot = sV + stv * C::kPair;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint32_t acc = (u > 0 || k > 0) ? 1u : 0u;
-            mma_bf16(gA, sdesc(base + k * 2048, 8192, 1024), sdesc(base + C::kTile + k * 2048, 8192, 1024),
-                     idG, acc);
-            mma_bf16(gB, sdesc(base + 2 * C::kTile + k * 2048, 8192, 1024),
-                     sdesc(base + 3 * C::kTile + k * 2048, 8192, 1024), idG, acc);
+            mma_bf16(gA, sdesc(kslot + k * 2048, 8192, 1024), sdesc(vslot + k * 2048, 8192, 1024), idG, acc);
+            mma_bf16(gB, sdesc(kslot + C::kTile + k * 2048, 8192, 1024),
+                     sdesc(vslot + C::kTile + k * 2048, 8192, 1024), idG, acc);
           }
-          mma_commit(bar(bKvEmpty0 + st));
+          mma_commit(bar(bKEmpty0 + stk));
+          mma_commit(bar(bVEmpty0 + stv));
         }
       }
       mma_commit(bar(bTailDone));
@@ -277,10 +325,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_bf16(tb + C::cNum, sdesc(sQA + off, 16, 1024), sdesc(sHA + k * 2048, D * 128, 1024), idN,
+          mma_bf16(tb + C::cNum, sdesc(sQA + off, 16, 1024), sdesc(sHA + k * 2048, D * 128, 1024), idN, k > 0);
+          mma_bf16(tb + laneB + C::cNum, sdesc(sQB + off, 16, 1024), sdesc(sHB + k * 2048, D * 128, 1024), idN,
                    k > 0);
-          mma_bf16(tb + laneB + C::cNum, sdesc(sQB + off, 16, 1024), sdesc(sHB + k * 2048, D * 128, 1024),
-                   idN, k > 0);
         }
         mma_commit(bar(bNumFull));
       }
@@ -292,8 +339,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
           mma_bf16(tb + C::cY, sdesc(sOlA + off, 16, 1024), sdesc(sW + k * 2048, D * 128, 1024), idN, k > 0);
-          mma_bf16(tb + laneB + C::cY, sdesc(sOlB + off, 16, 1024), sdesc(sW + k * 2048, D * 128, 1024),
-                   idN, k > 0);
+          mma_bf16(tb + laneB + C::cY, sdesc(sOlB + off, 16, 1024), sdesc(sW + k * 2048, D * 128, 1024), idN,
+                   k > 0);
         }
         mma_commit(bar(bYFull));
       }
@@ -310,11 +357,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     const int grow = blk * 64 + r;          // row inside the head
     const bool store_row = grow < N && (!isB || validB);
     const uint32_t tq = tb + (uint32_t(32 * warp) << 16);  // this warp's TMEM lane quarter
-    unsigned char* Prow = smem + (isB ? C::oPB : C::oPA) + r * 128;
-    const int32_t* mycrit = isB ? critB : critA;
+    unsigned char* Pbase = smem + C::oP + (isB ? 8192 : 0) + r * 128;
     const float sl2 = a.scale_log2;
+    // Only the block holding the last (partial) rows of the sequence has pad
+    // keys; the lists are ascending, so it can only be the last step.
+    const int jlast = dense ? Nb - 1 : checked((isB ? critB : critA)[nA - 1]);
+    const bool mask_last = jlast * 64 + 64 > N;
     float m = -INFINITY, l = 0.0f;
-    int pv_seen = -1;  // last step whose PV completion this thread has observed
 
     for (int t = 0; t < nA; ++t) {
       const int b = t & 1;
@@ -334,22 +383,24 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       }
       tc_fence_before();
       mbar_arrive(bar(bSFree0 + b));
-      const int j = crit_block(mycrit, t);
-      if (j * 64 + 64 > N) {
+      if (t == nA - 1 && mask_last) {
 #pragma unroll
         for (int i = 0; i < 64; ++i)
-          if (j * 64 + i >= N) s[i] = -INFINITY;
+          if (jlast * 64 + i >= N) s[i] = -INFINITY;
       }
-      float mx = -INFINITY;
+      float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
-      mx *= sl2;
+      for (int g = 0; g < 8; ++g) mx8[g] = s[g];
+#pragma unroll
+      for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
       if (t == 0) {
         m = mx;
       } else if (__any_sync(0xffffffffu, mx > m + 8.0f)) {
         // some row of this warp grew by more than 2^8: rescale the warp's O rows in TMEM
-        wait_w(bPvDone, (t - 1) & 1);
-        pv_seen = t - 1;
+        // once PV(t-1) has landed in O
+        wait_w(bPvDone0 + ((t - 1) & 1), ((t - 1) >> 1) & 1);
         tc_fence_after();
         const float mnew = fmaxf(m, mx);
         const float corr = ex2(m - mnew);
@@ -367,44 +418,64 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         tmem_wait_st();
       }
       uint32_t pk[32];
-      float sum = 0.0f;
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float p0 = ex2(fmaf(s[2 * i], sl2, -m));
         const float p1 = ex2(fmaf(s[2 * i + 1], sl2, -m));
-        sum += p0 + p1;
+        sum8[i & 7] += p0 + p1;
         pk[i] = pack_bf16(p0, p1);
       }
-      l += sum;
-      if (t > 0 && pv_seen != t - 1) {  // P buffer is free once PV(t-1) has completed
-        wait(bPvDone, (t - 1) & 1);
-        pv_seen = t - 1;
-      }
+      l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      // P buffer b is free once PV(t-2) has completed
+      if (t >= 2) wait(bPvDone0 + b, ((t >> 1) & 1) ^ 1);
+      unsigned char* Prow = Pbase + b * 16384;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(Prow + (uint32_t(c ^ (r & 7)) << 4)) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(bPFull));
+      mbar_arrive(bar(bPFull0 + b));
     }
-    if (nA > 0 && pv_seen != nA - 1) wait_w(bPvDone, (nA - 1) & 1);
+    // final O: the last PV (and every earlier product) has completed
+    wait_w(bPvDone0 + ((nA - 1) & 1), ((nA - 1) >> 1) & 1);
     tc_fence_after();
     const float inv_l = 1.0f / l;
 
     float den = 1.0f;
     if (has_marg) {
-      // Z_i = Z_tot - sum over the excluded blocks of z_j, for blocks A and B
+      // Z_i = Z_tot - sum over the excluded blocks of z_j, blocks A and B.
+      // Thread handles (X, c) for e = tid and tid + 128 < 2D; block indices are
+      // fetched 32 at a time, one per lane, and broadcast.
       const float* zt = a.ztot + size_t(bh) * D;
       const float* zb = a.zblk + size_t(bh) * Nb * D;
-      for (int e = tid; e < 2 * D; e += 128) {
-        const int X = e / D, c = e % D;
-        const int32_t* cl = X ? critB : critA;
-        const int32_t* nl = X ? negB : negA;
-        float z = zt[c];
-        for (int u = 0; u < nE; ++u) z -= zb[size_t(excl_block(cl, nl, u)) * D + c];
-        zs[X][c] = z;
+      float z[2];
+      int zc[2], zx[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = tid + 128 * k;
+        zx[k] = e / D;
+        zc[k] = e % D;
+        z[k] = e < 2 * D ? zt[zc[k]] : 0.0f;
       }
+      for (int u0 = 0; u0 < nE; u0 += 32) {
+        const int uu = u0 + lane;
+        const int myA = uu < nE ? step_block(0, nA + uu) : 0;
+        const int myB = uu < nE ? step_block(1, nA + uu) : 0;
+        const int cnt = min(32, nE - u0);
+#pragma unroll 4
+        for (int i = 0; i < cnt; ++i) {
+          const int jA = __shfl_sync(0xffffffffu, myA, i);
+          const int jB = __shfl_sync(0xffffffffu, myB, i);
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+            if (tid + 128 * k < 2 * D) z[k] -= zb[size_t(zx[k] ? jB : jA) * D + zc[k]];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (tid + 128 * k < 2 * D) zs[zx[k]][zc[k]] = z[k];
       // phi(Q) of this row, in place of Q (K-major swizzled tile); three passes
       // over shared memory (max, sum, write) keep the row out of registers
       unsigned char* Qrow = smem + (isB ? C::oQB : C::oQA);
@@ -446,48 +517,31 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       wait_w(bTailDone, 0);
       tc_fence_after();
       const float* ht = a.htot32 + size_t(bh) * D * D;
-      if (D == 128) {
+      // D=128: G rows c = TMEM lanes (M = 128), G_A and G_B in separate columns;
+      // D=64:  G_A rows in lanes 0-15 of each quarter, G_B in lanes 16-31.
+      const int c = D == 128 ? tid : r;
+      constexpr int kBlocksPerThread = D == 128 ? 2 : 1;
 #pragma unroll 1
-        for (int X = 0; X < 2; ++X) {
-          const int c = tid;  // TMEM lane = row c of G (M = 128)
-          const uint32_t tg = tq + C::cG + X * 128;
-          unsigned char* Hrow = smem + (X ? C::oHB : C::oHA);
-#pragma unroll 1
-          for (int ch = 0; ch < D / 32; ++ch) {
-            float g[32];
-            tmem_ld32(tg + ch * 32, g);
-            tmem_wait_ld();
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float4 hv[8];
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-              const int e0 = ch * 32 + q8 * 8;
-              const float4 h0 = *reinterpret_cast<const float4*>(ht + size_t(c) * D + e0);
-              const float4 h1 = *reinterpret_cast<const float4*>(ht + size_t(c) * D + e0 + 4);
-              const uint4 v = make_uint4(pack_bf16(h0.x - g[q8 * 8 + 0], h0.y - g[q8 * 8 + 1]),
-                                         pack_bf16(h0.z - g[q8 * 8 + 2], h0.w - g[q8 * 8 + 3]),
-                                         pack_bf16(h1.x - g[q8 * 8 + 4], h1.y - g[q8 * 8 + 5]),
-                                         pack_bf16(h1.z - g[q8 * 8 + 6], h1.w - g[q8 * 8 + 7]));
-              *reinterpret_cast<uint4*>(Hrow + (e0 >> 6) * (D * 128) + sw128_chunk(c, (e0 & 63) >> 3)) = v;
-            }
-          }
-        }
-      } else {
-        const int c = r;  // M = 64 layout: block A rows in lanes 0-15, block B in 16-31
-        unsigned char* Hrow = smem + (isB ? C::oHB : C::oHA);
-#pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int q = 0; q < 8; ++q) hv[q] = *reinterpret_cast<const float4*>(ht + size_t(c) * D + ch * 32 + 4 * q);
+#pragma unroll
+        for (int X = 0; X < kBlocksPerThread; ++X) {
+          const bool xb = D == 128 ? X == 1 : isB;
           float g[32];
-          tmem_ld32(tq + C::cG + ch * 32, g);
+          tmem_ld32(tq + C::cG + (D == 128 ? X * 128 : 0) + ch * 32, g);
           tmem_wait_ld();
+          unsigned char* Hbase = smem + (xb ? C::oHB : C::oHA);
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             const int e0 = ch * 32 + q8 * 8;
-            const float4 h0 = *reinterpret_cast<const float4*>(ht + size_t(c) * D + e0);
-            const float4 h1 = *reinterpret_cast<const float4*>(ht + size_t(c) * D + e0 + 4);
+            const float4 h0 = hv[2 * q8], h1 = hv[2 * q8 + 1];
             const uint4 v = make_uint4(pack_bf16(h0.x - g[q8 * 8 + 0], h0.y - g[q8 * 8 + 1]),
                                        pack_bf16(h0.z - g[q8 * 8 + 2], h0.w - g[q8 * 8 + 3]),
                                        pack_bf16(h1.x - g[q8 * 8 + 4], h1.y - g[q8 * 8 + 5]),
                                        pack_bf16(h1.z - g[q8 * 8 + 6], h1.w - g[q8 * 8 + 7]));
-            *reinterpret_cast<uint4*>(Hrow + (e0 >> 6) * (D * 128) + sw128_chunk(c, (e0 & 63) >> 3)) = v;
+            *reinterpret_cast<uint4*>(Hbase + (e0 >> 6) * (D * 128) + sw128_chunk(c, (e0 & 63) >> 3)) = v;
           }
         }
       }

@@ -11,15 +11,18 @@
 // The per-query-block sums over marginal blocks are formed later as
 // H_i = H_tot - sum_{j excluded from row i} h_j (likewise Z_i), with the
 // excluded (critical and negligible) blocks' terms recomputed from the tiles
-// the attention kernel loads, so H_tot / Z_tot are all that is stored here.
-// Reductions run in a fixed order (no atomics): results are deterministic.
+// the attention kernel loads, so H_tot / Z_tot and z_j are all that is stored
+// here besides phi(K). Reductions run in a fixed order (no atomics): results
+// are deterministic.
 #include "sla_internal.cuh"
 
 namespace sla {
 
-// CTA of 256 threads (8 warps) per (1024-token chunk, head). For each 64-token
-// block: phi(K) rows -> global (bf16) and shared memory, z_j -> global,
-// H_chunk += phi(K_j)^T V_j on tensor cores (mma.sync m16n8k16, fp32 acc).
+// CTA of 256 threads (8 warps) per (1024-token chunk, head). The K and V
+// tiles of the next 64-token block stream in (cp.async, double-buffered)
+// while the current one is processed: phi(K) rows -> shared memory and global
+// (bf16), z_j -> global, H_chunk += phi(K_j)^T V_j on tensor cores
+// (mma.sync m16n8k16, fp32 accumulation).
 template <int D>
 __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __restrict__ K,
                                                       const __nv_bfloat16* __restrict__ V,
@@ -27,12 +30,15 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
                                                       float* __restrict__ zblk,
                                                       float* __restrict__ hpart, int N, int Npad,
                                                       int Nb, int nchunk) {
-  constexpr int CPR = D / 8;            // 16-byte chunks per row
-  constexpr int WPM = 128 / D;          // warps per 16-row m tile (1 for D=128, 2 for D=64)
-  constexpr int NCOL = D / WPM;         // output columns per warp
-  constexpr int NT = NCOL / 8;          // n tiles per warp
-  __shared__ __align__(128) __nv_bfloat16 PK[64 * D];
-  __shared__ __align__(128) __nv_bfloat16 Vs[64 * D];
+  constexpr int CPR = D / 8;    // 16-byte chunks per row
+  constexpr int WPM = 128 / D;  // warps per 16-row m tile (1 for D=128, 2 for D=64)
+  constexpr int NCOL = D / WPM; // output columns per warp
+  constexpr int NT = NCOL / 8;  // n tiles per warp
+  constexpr int kT = 64 * D;    // elements of a 64-row tile
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [2][64 x D]
+  __nv_bfloat16* Vs = Ks + 2 * kT;                                  // [2][64 x D]
+  __nv_bfloat16* PK = Vs + 2 * kT;                                  // [64 x D]
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mt = warp / WPM, n0 = (warp % WPM) * NCOL;
@@ -40,37 +46,57 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
   const int jb0 = chunk * (kHzChunk / kBlock);
   const int jb1 = min(Nb, jb0 + kHzChunk / kBlock);
 
+  auto load_block = [&](int jb, int buf) {
+    const int t0 = jb * kBlock;
+    const int nv = min(kBlock, N - t0);
+    for (int id = threadIdx.x; id < 64 * CPR; id += 256) {
+      const int r = id / CPR, ch = id % CPR;
+      const bool v = r < nv;  // rows past N are zero-filled, never read
+      const size_t g = hoff + size_t(t0 + r) * D + ch * 8;
+      const int s = r * D + ((ch ^ (r & 7)) << 3);
+      cp_async16(smem_u32(Ks + buf * kT + s), v ? (const void*)(K + g) : (const void*)K, v);
+      cp_async16(smem_u32(Vs + buf * kT + s), v ? (const void*)(V + g) : (const void*)V, v);
+    }
+  };
+
   float acc[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[t][e] = 0.0f;
 
+  load_block(jb0, 0);
+  cp_async_commit();
   for (int jb = jb0; jb < jb1; ++jb) {
+    const int buf = (jb - jb0) & 1;
     const int t0 = jb * kBlock;
     const int nv = min(kBlock, N - t0);
-    // V tile (rows >= N zero-filled)
-    for (int id = threadIdx.x; id < 64 * CPR; id += 256) {
-      const int r = id / CPR, ch = id % CPR;
-      const bool v = r < nv;
-      cp_async16(smem_u32(Vs + r * D + ((ch ^ (r & 7)) << 3)),
-                 v ? (const void*)(V + hoff + size_t(t0 + r) * D + ch * 8) : (const void*)V, v);
-    }
+    if (jb + 1 < jb1) load_block(jb + 1, buf ^ 1);
     cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
     // phi(K) rows: warp w handles rows w, w+8, ...; a lane holds D/32 columns
+    const __nv_bfloat16* Kb = Ks + buf * kT;
+    constexpr int PL = D / 32;
+    const int col = lane * PL;
     for (int r = warp; r < 64; r += 8) {
-      constexpr int PL = D / 32;
       float x[PL];
-      const int col = lane * PL;
-      __nv_bfloat16* gdst = phik + hoff + size_t(t0 + r) * D + col;
       if (r < nv) {
-        const __nv_bfloat16* src = K + hoff + size_t(t0 + r) * D + col;
-        float m = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < PL; ++e) {
-          x[e] = bf2f(src[e]);
-          m = fmaxf(m, x[e]);
+        const __nv_bfloat16* src = Kb + swz(r, col, D);
+        if constexpr (PL == 4) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(src);
+          x[0] = bf16_lo(raw.x);
+          x[1] = bf16_hi(raw.x);
+          x[2] = bf16_lo(raw.y);
+          x[3] = bf16_hi(raw.y);
+        } else {
+          const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
+          x[0] = bf16_lo(raw);
+          x[1] = bf16_hi(raw);
         }
+        float m = x[0];
+#pragma unroll
+        for (int e = 1; e < PL; ++e) m = fmaxf(m, x[e]);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
         float s = 0.0f;
@@ -92,6 +118,7 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
 #pragma unroll
       for (int e = 0; e < PL / 2; ++e) pk[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
       __nv_bfloat16* sdst = PK + swz(r, col, D);
+      __nv_bfloat16* gdst = phik + hoff + size_t(t0 + r) * D + col;
       if constexpr (PL == 4) {
         *reinterpret_cast<uint2*>(sdst) = make_uint2(pk[0], pk[1]);
         *reinterpret_cast<uint2*>(gdst) = make_uint2(pk[0], pk[1]);
@@ -100,7 +127,6 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
         *reinterpret_cast<uint32_t*>(gdst) = pk[0];
       }
     }
-    cp_async_wait<0>();
     __syncthreads();
     // z_j: column sums of the (bf16) phi values, rows ascending
     if (threadIdx.x < D) {
@@ -110,6 +136,7 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
       zblk[(size_t(bh) * Nb + jb) * D + c] = z;
     }
     // H_chunk += phi(K_j)^T V_j : A = phi(K)^T (m = dim, k = token), B = V
+    const __nv_bfloat16* Vb = Vs + buf * kT;
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t a[4];
@@ -123,7 +150,7 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
         uint32_t b0, b1, b2, b3;
         const int tr = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
         const int tc = n0 + 16 * q + ((lane >> 4) << 3);
-        ldsm_x4_t(smem_u32(Vs + swz(tr, tc, D)), b0, b1, b2, b3);
+        ldsm_x4_t(smem_u32(Vb + swz(tr, tc, D)), b0, b1, b2, b3);
         mma16816(acc[2 * q], a, b0, b1);
         mma16816(acc[2 * q + 1], a, b2, b3);
       }
@@ -141,14 +168,22 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
   }
 }
 
+template <int D>
+static cudaError_t launch_hz_t(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                               __nv_bfloat16* phik, float* zblk, float* hpart, cudaStream_t s) {
+  const int bytes = 5 * 64 * D * 2;
+  cudaError_t e =
+      cudaFuncSetAttribute(phik_hz_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  phik_hz_kernel<D><<<dim3(L.nchunk, L.BH), 256, bytes, s>>>(K, V, phik, zblk, hpart, L.N, L.Npad, L.Nb,
+                                                            L.nchunk);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                            __nv_bfloat16* phik, float* zblk, float* hpart, cudaStream_t s) {
-  dim3 grid(L.nchunk, L.BH);
-  if (L.d == 128)
-    phik_hz_kernel<128><<<grid, 256, 0, s>>>(K, V, phik, zblk, hpart, L.N, L.Npad, L.Nb, L.nchunk);
-  else
-    phik_hz_kernel<64><<<grid, 256, 0, s>>>(K, V, phik, zblk, hpart, L.N, L.Npad, L.Nb, L.nchunk);
-  return cudaGetLastError();
+  return L.d == 128 ? launch_hz_t<128>(L, K, V, phik, zblk, hpart, s)
+                    : launch_hz_t<64>(L, K, V, phik, zblk, hpart, s);
 }
 
 // H_tot = sum over chunks (ascending); Z_tot = sum over blocks (ascending).
