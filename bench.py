@@ -77,7 +77,7 @@ def correction_flops(w):
 def stage_bytes(w):
     """Bytes each memory-bound stage moves (reads + writes) in this design."""
     BH, N, Np, Nb, d = w.B * w.H, w.N, w.N_pad, w.Nb, w.d
-    nchunk = (Np + 1023) // 1024
+    nchunk = (Np + 511) // 512
     return {
         "pool": BH * (2 * N * d * 2 + 2 * Nb * d * 4),
         "phik_hz": BH * (2 * N * d * 2 + Np * d * 2 + Nb * d * 4 + nchunk * d * d * 4),

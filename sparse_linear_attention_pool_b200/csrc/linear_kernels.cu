@@ -28,7 +28,8 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
                                                       const __nv_bfloat16* __restrict__ V,
                                                       __nv_bfloat16* __restrict__ phik,
                                                       float* __restrict__ zblk,
-                                                      float* __restrict__ hpart, int N, int Npad,
+                                                      float* __restrict__ hpart, float* __restrict__ zpart,
+                                                      int N, int Npad,
                                                       int Nb, int nchunk) {
   constexpr int CPR = D / 8;    // 16-byte chunks per row
   constexpr int WPM = 128 / D;  // warps per 16-row m tile (1 for D=128, 2 for D=64)
@@ -64,6 +65,7 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
   for (int t = 0; t < NT; ++t)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[t][e] = 0.0f;
+  float zsum[2] = {0.0f, 0.0f};
 
   load_block(jb0, 0);
   cp_async_commit();
@@ -128,15 +130,11 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
       }
     }
     __syncthreads();
-    // z_j: column sums of the (bf16) phi values, rows ascending
-    if (threadIdx.x < D) {
-      const int c = threadIdx.x;
-      float z = 0.0f;
-      for (int r = 0; r < 64; ++r) z += bf2f(PK[swz(r, c, D)]);
-      zblk[(size_t(bh) * Nb + jb) * D + c] = z;
-    }
-    // H_chunk += phi(K_j)^T V_j : A = phi(K)^T (m = dim, k = token), B = V
+    // H_chunk += phi(K_j)^T V_j : A = phi(K)^T (m = dim, k = token), B = V.
+    // z_j = phi(K_j)^T 1 rides along as one more n-tile with B = all ones.
     const __nv_bfloat16* Vb = Vs + buf * kT;
+    float zacc[4] = {0.f, 0.f, 0.f, 0.f};
+    constexpr uint32_t kOnes = 0x3F803F80u;  // bf16x2 (1.0, 1.0)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t a[4];
@@ -145,6 +143,7 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
         const int tc = 16 * mt + (((lane >> 3) & 1) << 3);
         ldsm_x4_t(smem_u32(PK + swz(tr, tc, D)), a[0], a[1], a[2], a[3]);
       }
+      if (n0 == 0) mma16816(zacc, a, kOnes, kOnes);
 #pragma unroll
       for (int q = 0; q < NT / 2; ++q) {
         uint32_t b0, b1, b2, b3;
@@ -155,7 +154,19 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
         mma16816(acc[2 * q + 1], a, b2, b3);
       }
     }
+    if (n0 == 0 && (lane & 3) == 0) {  // every column of the ones-tile holds the row sum
+      float* zdst = zblk + (size_t(bh) * Nb + jb) * D + 16 * mt + (lane >> 2);
+      zdst[0] = zacc[0];
+      zdst[8] = zacc[2];
+      zsum[0] += zacc[0];  // chunk partial of Z_tot, blocks in ascending order
+      zsum[1] += zacc[2];
+    }
     __syncthreads();
+  }
+  if (n0 == 0 && (lane & 3) == 0) {
+    float* zdst = zpart + (size_t(bh) * nchunk + chunk) * D + 16 * mt + (lane >> 2);
+    zdst[0] = zsum[0];
+    zdst[8] = zsum[1];
   }
   // partial H of this chunk: rows (dims) 16 mt + lane/4 (+8), columns n0 + 8t + 2(lane%4)
   float* hp = hpart + (size_t(bh) * nchunk + chunk) * D * D;
@@ -170,49 +181,61 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
 
 template <int D>
 static cudaError_t launch_hz_t(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                               __nv_bfloat16* phik, float* zblk, float* hpart, cudaStream_t s) {
+                               __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
+                               cudaStream_t s) {
   const int bytes = 5 * 64 * D * 2;
   cudaError_t e =
       cudaFuncSetAttribute(phik_hz_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  phik_hz_kernel<D><<<dim3(L.nchunk, L.BH), 256, bytes, s>>>(K, V, phik, zblk, hpart, L.N, L.Npad, L.Nb,
-                                                            L.nchunk);
+  phik_hz_kernel<D><<<dim3(L.nchunk, L.BH), 256, bytes, s>>>(K, V, phik, zblk, hpart, zpart, L.N, L.Npad,
+                                                            L.Nb, L.nchunk);
   return cudaGetLastError();
 }
 
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                           __nv_bfloat16* phik, float* zblk, float* hpart, cudaStream_t s) {
-  return L.d == 128 ? launch_hz_t<128>(L, K, V, phik, zblk, hpart, s)
-                    : launch_hz_t<64>(L, K, V, phik, zblk, hpart, s);
+                           __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
+                           cudaStream_t s) {
+  return L.d == 128 ? launch_hz_t<128>(L, K, V, phik, zblk, hpart, zpart, s)
+                    : launch_hz_t<64>(L, K, V, phik, zblk, hpart, zpart, s);
 }
 
-// H_tot = sum over chunks (ascending); Z_tot = sum over blocks (ascending).
-__global__ void __launch_bounds__(256) hz_reduce_kernel(const float* __restrict__ zblk,
+// Fixed-order sum of n strided values: 8 interleaved partial sums (element i
+// goes to partial i % 8), combined pairwise. Independent loads keep the
+// memory pipe busy; the order is the same on every call.
+__device__ __forceinline__ float strided_sum(const float* __restrict__ src, int n, size_t stride) {
+  float p[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int i = 0;
+  for (; i + 8 <= n; i += 8) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) p[k] += src[size_t(i + k) * stride];
+  }
+  for (int k = 0; i < n; ++i, ++k) p[k] += src[size_t(i) * stride];
+  return ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+}
+
+// H_tot and Z_tot = sums of the per-chunk partials (fixed order, see
+// strided_sum). Blocks x < d*d/256 reduce H; the last block reduces Z.
+__global__ void __launch_bounds__(256) hz_reduce_kernel(const float* __restrict__ zpart,
                                                         const float* __restrict__ hpart,
                                                         float* __restrict__ htot32,
-                                                        float* __restrict__ ztot, int Nb, int nchunk,
-                                                        int d) {
+                                                        float* __restrict__ ztot, int nchunk, int d) {
   const int bh = blockIdx.y;
-  const int e = blockIdx.x * 256 + threadIdx.x;
   const size_t dd = size_t(d) * d;
-  if (e < int(dd)) {
-    const float* src = hpart + size_t(bh) * nchunk * dd + e;
-    float s = 0.0f;
-    for (int c = 0; c < nchunk; ++c) s += src[size_t(c) * dd];
-    htot32[size_t(bh) * dd + e] = s;
-  }
-  if (blockIdx.x == 0 && threadIdx.x < d) {
-    const float* zs = zblk + size_t(bh) * Nb * d + threadIdx.x;
-    float s = 0.0f;
-    for (int j = 0; j < Nb; ++j) s += zs[size_t(j) * d];
-    ztot[size_t(bh) * d + threadIdx.x] = s;
+  const int nh = int((dd + 255) / 256);
+  if (int(blockIdx.x) < nh) {
+    const int e = blockIdx.x * 256 + threadIdx.x;
+    if (e < int(dd))
+      htot32[size_t(bh) * dd + e] = strided_sum(hpart + size_t(bh) * nchunk * dd + e, nchunk, dd);
+  } else if (threadIdx.x < d) {
+    ztot[size_t(bh) * d + threadIdx.x] =
+        strided_sum(zpart + size_t(bh) * nchunk * d + threadIdx.x, nchunk, size_t(d));
   }
 }
 
-cudaError_t launch_hz_reduce(const Layout& L, const float* zblk, const float* hpart, float* htot32,
+cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* hpart, float* htot32,
                              float* ztot, cudaStream_t s) {
-  dim3 grid((L.d * L.d + 255) / 256, L.BH);
-  hz_reduce_kernel<<<grid, 256, 0, s>>>(zblk, hpart, htot32, ztot, L.Nb, L.nchunk, L.d);
+  dim3 grid((L.d * L.d + 255) / 256 + 1, L.BH);
+  hz_reduce_kernel<<<grid, 256, 0, s>>>(zpart, hpart, htot32, ztot, L.nchunk, L.d);
   return cudaGetLastError();
 }
 

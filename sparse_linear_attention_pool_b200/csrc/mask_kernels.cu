@@ -111,41 +111,46 @@ cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bflo
 // ---------------------------------------------------------------------------
 // pooled scores
 // ---------------------------------------------------------------------------
-// CTA: 16 x 16 threads, a 64 x 64 tile of S; thread (tx, ty) owns rows
-// ty + 16a and columns tx + 16b. k runs ascending across 32-wide chunks.
+// CTA: 16 x 16 threads, a 64 x 128 tile of S; thread (tx, ty) owns rows
+// ty + 16a (a < 4) and columns tx + 16b (b < 8). k runs ascending across
+// 32-wide chunks.
 __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ qbar,
                                                      const float* __restrict__ kbar,
                                                      float* __restrict__ S, int Nb, int d) {
   __shared__ float Qs[64][33];
-  __shared__ float Ks[64][33];
+  __shared__ float Ks[128][33];
   const int tx = threadIdx.x, ty = threadIdx.y, tid = ty * 16 + tx;
-  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64, bh = blockIdx.z;
+  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 128, bh = blockIdx.z;
   const float* qb = qbar + size_t(bh) * Nb * d;
   const float* kb = kbar + size_t(bh) * Nb * d;
-  float acc[4][4];
+  float acc[4][8];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
   for (int k0 = 0; k0 < d; k0 += 32) {
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
       const int r = it * 8 + tid / 32, c = tid % 32;
       Qs[r][c] = (i0 + r < Nb) ? qb[size_t(i0 + r) * d + k0 + c] : 0.0f;
+    }
+#pragma unroll
+    for (int it = 0; it < 16; ++it) {
+      const int r = it * 8 + tid / 32, c = tid % 32;
       Ks[r][c] = (j0 + r < Nb) ? kb[size_t(j0 + r) * d + k0 + c] : 0.0f;
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
     for (int kk = 0; kk < 32; ++kk) {
-      float qv[4], kv[4];
+      float qv[4], kv[8];
 #pragma unroll
       for (int a = 0; a < 4; ++a) qv[a] = Qs[ty + 16 * a][kk];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) kv[b] = Ks[tx + 16 * b][kk];
+      for (int b = 0; b < 8; ++b) kv[b] = Ks[tx + 16 * b][kk];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(qv[a], kv[b]));
+        for (int b = 0; b < 8; ++b) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(qv[a], kv[b]));
     }
     __syncthreads();
   }
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
     const int i = i0 + ty + 16 * a;
     if (i >= Nb) continue;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
+    for (int b = 0; b < 8; ++b) {
       const int j = j0 + tx + 16 * b;
       if (j < Nb) Sb[size_t(i) * Nb + j] = acc[a][b];
     }
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
 
 cudaError_t launch_scores(const Layout& L, const float* qbar, const float* kbar, float* scores,
                           cudaStream_t s) {
-  dim3 grid((L.Nb + 63) / 64, (L.Nb + 63) / 64, L.BH);
+  dim3 grid((L.Nb + 127) / 128, (L.Nb + 63) / 64, L.BH);
   scores_kernel<<<grid, dim3(16, 16), 0, s>>>(qbar, kbar, scores, L.Nb, L.d);
   return cudaGetLastError();
 }
@@ -172,7 +177,10 @@ cudaError_t launch_scores(const Layout& L, const float* qbar, const float* kbar,
 // ---------------------------------------------------------------------------
 // classification
 // ---------------------------------------------------------------------------
-constexpr int kClsThreads = 256;
+// One warp per row (bh, query block i); 8 rows per CTA. The row's keys and a
+// 256-bin histogram live in the warp's slice of shared memory; everything is
+// warp-synchronous.
+constexpr int kClsWarps = 8;
 
 // Monotone map float -> uint32 (larger float, larger key); -0 and +0 map alike.
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -180,148 +188,123 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive prefix sum of `v` over the CTA's threads in thread order.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += t;
-  }
-  if (lane == 31) warp_tot[wid] = incl;
-  __syncthreads();
-  int base = 0;
-  for (int w = 0; w < wid; ++w) base += warp_tot[w];
-  __syncthreads();
-  return base + incl - v;
-}
-
-// k-th largest key (k >= 1) by 4 passes of an 8-bit radix select. Returns the
-// key value T and `need`, the number of elements equal to T that belong to
-// the top k (the others above T are all in it).
-__device__ void radix_select_top(const uint32_t* keys, int lo, int hi, int k, int* hist, int* sel,
-                                 uint32_t& T, int& need) {
+// k-th largest key (1 <= k <= n) by 4 passes of an 8-bit radix select. Returns
+// the key value T and `need`, the number of elements equal to T that belong to
+// the top k (every element above T is in it).
+__device__ void warp_select_top(const uint32_t* keys, int n, int k, int* hist, uint32_t& T, int& need) {
+  const int lane = threadIdx.x & 31;
   uint32_t prefix = 0, pmask = 0;
   int rem = k;
-  const int tid = threadIdx.x, lane = tid & 31;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    hist[tid] = 0;  // kClsThreads == 256 bins
-    __syncthreads();
-    for (int j = lo; j < hi; ++j) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
       const uint32_t key = keys[j];
       if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
-    __syncthreads();
-    if (tid < 32) {
-      int c[8], sum = 0;
+    __syncwarp();
+    // lane l scans bins 255-8l down to 248-8l (largest digits first)
+    int c[8], sum = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = hist[255 - 8 * lane - e];
+      sum += c[e];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= rem);
+    const int src = __ffs(hit) - 1;  // hit != 0: the total count n >= rem
+    int sel = 0, nrem = 0;
+    if (lane == src) {
+      int cum = incl - sum;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        c[e] = hist[255 - 8 * lane - e];
-        sum += c[e];
-      }
-      int incl = sum;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += t;
-      }
-      const unsigned hit = __ballot_sync(0xffffffffu, incl >= rem);
-      if (lane == __ffs(hit) - 1) {
-        int cum = incl - sum;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (cum + c[e] >= rem) {
-            sel[0] = 255 - 8 * lane - e;
-            sel[1] = rem - cum;
-            break;
-          }
-          cum += c[e];
+        if (cum + c[e] >= rem) {
+          sel = 255 - 8 * lane - e;
+          nrem = rem - cum;
+          break;
         }
+        cum += c[e];
       }
     }
-    __syncthreads();
-    prefix |= uint32_t(sel[0]) << shift;
+    sel = __shfl_sync(0xffffffffu, sel, src);
+    rem = __shfl_sync(0xffffffffu, nrem, src);
+    prefix |= uint32_t(sel) << shift;
     pmask |= 0xFFu << shift;
-    rem = sel[1];
-    __syncthreads();
+    __syncwarp();
   }
   T = prefix;
   need = rem;
 }
 
-// One CTA per (bh, query block i). Top k_crit by (score desc, index asc) are
-// critical; elements outside the top (Nb - k_neg) are negligible.
-__global__ void __launch_bounds__(kClsThreads) classify_kernel(const float* __restrict__ S,
-                                                               int8_t* __restrict__ Mc,
-                                                               int32_t* __restrict__ crit,
-                                                               int32_t* __restrict__ neg, int Nb,
-                                                               int kc, int kn) {
-  __shared__ uint32_t keys[SLA_MAX_BLOCKS];
-  __shared__ int hist[256];
-  __shared__ int sel[2];
-  __shared__ int warp_tot[kClsThreads / 32];
-  const size_t row = size_t(blockIdx.y) * Nb + blockIdx.x;
+// Top k_crit by (score desc, index asc) are critical; elements outside the
+// top (Nb - k_neg) are negligible.
+__global__ void __launch_bounds__(32 * kClsWarps) classify_kernel(const float* __restrict__ S,
+                                                                  int8_t* __restrict__ Mc,
+                                                                  int32_t* __restrict__ crit,
+                                                                  int32_t* __restrict__ neg, int Nb,
+                                                                  int kc, int kn, int rows) {
+  extern __shared__ uint32_t cls_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row_i = blockIdx.x * kClsWarps + warp;
+  if (row_i >= rows) return;  // whole warp
+  uint32_t* keys = cls_smem + size_t(warp) * (Nb + 256);
+  int* hist = reinterpret_cast<int*>(keys + Nb);
+  const size_t row = size_t(row_i);
   const float* srow = S + row * Nb;
-  const int E = (Nb + kClsThreads - 1) / kClsThreads;
-  const int lo = min(Nb, int(threadIdx.x) * E), hi = min(Nb, lo + E);
-  for (int j = threadIdx.x; j < Nb; j += kClsThreads) keys[j] = order_key(srow[j]);
-  __syncthreads();
+  for (int j = lane; j < Nb; j += 32) keys[j] = order_key(srow[j]);
+  __syncwarp();
 
-  // top k_crit
-  uint32_t Tc;
-  int needc;
-  radix_select_top(keys, lo, hi, kc, hist, sel, Tc, needc);
-  int eq = 0;
-  for (int j = lo; j < hi; ++j) eq += keys[j] == Tc;
-  int eqrank = block_exclusive_scan(eq, warp_tot);
-  // top (Nb - k_neg): everything else is negligible
-  uint32_t Tn = 0;
-  int needn = 0, eqrank_n = 0;
-  if (kn > 0) {
-    radix_select_top(keys, lo, hi, Nb - kn, hist, sel, Tn, needn);
-    int eqn = 0;
-    for (int j = lo; j < hi; ++j) eqn += keys[j] == Tn;
-    eqrank_n = block_exclusive_scan(eqn, warp_tot);
-  }
-  // labels
+  uint32_t Tc, Tn = 0;
+  int needc, needn = 0;
+  warp_select_top(keys, Nb, kc, hist, Tc, needc);
+  if (kn > 0) warp_select_top(keys, Nb, Nb - kn, hist, Tn, needn);
+
   int8_t* mrow = Mc + row * Nb;
-  int ncrit = 0, nneg = 0;
-  for (int j = lo; j < hi; ++j) {
-    const uint32_t key = keys[j];
-    bool c = key > Tc || (key == Tc && eqrank < needc);
-    eqrank += key == Tc;
-    bool n = false;
-    if (kn > 0) {
-      const bool top = key > Tn || (key == Tn && eqrank_n < needn);
-      eqrank_n += key == Tn;
-      n = !top;
-    }
-    mrow[j] = c ? int8_t(1) : (n ? int8_t(-1) : int8_t(0));
-    ncrit += c;
-    nneg += n;
-  }
-  // ascending index lists
-  int pc = block_exclusive_scan(ncrit, warp_tot);
-  int pn = block_exclusive_scan(nneg, warp_tot);
   int32_t* crow = crit + row * kc;
   int32_t* nrow = neg + row * (kn > 0 ? kn : 1);
-  for (int j = lo; j < hi; ++j) {
-    const int8_t m = mrow[j];
-    if (m == 1) {
-      if (pc < kc) crow[pc] = j;  // exactly k_crit labels exist; the bound is defensive
-      ++pc;
-    } else if (m == -1) {
-      if (pn < kn) nrow[pn] = j;
-      ++pn;
+  const unsigned lt = (1u << lane) - 1u;
+  int eqc_seen = 0, eqn_seen = 0, ncrit = 0, nneg = 0;
+  for (int base = 0; base < Nb; base += 32) {
+    const int j = base + lane;
+    const bool valid = j < Nb;
+    const uint32_t key = valid ? keys[j] : 0u;
+    const bool eqc = valid && key == Tc;
+    const unsigned eqc_mask = __ballot_sync(0xffffffffu, eqc);
+    const bool c = valid && (key > Tc || (eqc && eqc_seen + __popc(eqc_mask & lt) < needc));
+    eqc_seen += __popc(eqc_mask);
+    bool n = false;
+    if (kn > 0) {
+      const bool eqn = valid && key == Tn;
+      const unsigned eqn_mask = __ballot_sync(0xffffffffu, eqn);
+      const bool top = key > Tn || (eqn && eqn_seen + __popc(eqn_mask & lt) < needn);
+      eqn_seen += __popc(eqn_mask);
+      n = valid && !top;
     }
+    if (valid) mrow[j] = c ? int8_t(1) : (n ? int8_t(-1) : int8_t(0));
+    const unsigned cm = __ballot_sync(0xffffffffu, c);
+    const unsigned nm = __ballot_sync(0xffffffffu, n);
+    // exactly k_crit / k_neg labels exist; the bounds are defensive
+    const int pc = ncrit + __popc(cm & lt), pn = nneg + __popc(nm & lt);
+    if (c && pc < kc) crow[pc] = j;
+    if (n && pn < kn) nrow[pn] = j;
+    ncrit += __popc(cm);
+    nneg += __popc(nm);
   }
 }
 
 cudaError_t launch_classify(const Layout& L, const float* scores, int8_t* mc, int32_t* crit,
                             int32_t* neg, cudaStream_t s) {
-  dim3 grid(L.Nb, L.BH);
-  classify_kernel<<<grid, kClsThreads, 0, s>>>(scores, mc, crit, neg, L.Nb, L.kc, L.kn);
+  const int rows = L.BH * L.Nb;
+  const int bytes = kClsWarps * (L.Nb + 256) * 4;  // <= 8 * 4352 * 4 = 139264 for Nb <= 4096
+  cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  classify_kernel<<<(rows + kClsWarps - 1) / kClsWarps, 32 * kClsWarps, bytes, s>>>(
+      scores, mc, crit, neg, L.Nb, L.kc, L.kn, rows);
   return cudaGetLastError();
 }
 

@@ -97,6 +97,7 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   __nv_bfloat16* phik = reinterpret_cast<__nv_bfloat16*>(ws + L.phik);
   float* zblk = reinterpret_cast<float*>(ws + L.zblk);
   float* hpart = reinterpret_cast<float*>(ws + L.hpart);
+  float* zpart = reinterpret_cast<float*>(ws + L.zpart);
   float* htot32 = reinterpret_cast<float*>(ws + L.htot32);
   float* ztot = reinterpret_cast<float*>(ws + L.ztot);
   const bool sla2 = p->variant == SLA_VARIANT_SLA2;
@@ -115,9 +116,9 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   mark(2);
   if (e == cudaSuccess) e = launch_classify(L, scores, mc, crit, neg, s);
   mark(3);
-  if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, s);
+  if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, zpart, s);
   mark(4);
-  if (e == cudaSuccess) e = launch_hz_reduce(L, zblk, hpart, htot32, ztot, s);
+  if (e == cudaSuccess) e = launch_hz_reduce(L, zpart, hpart, htot32, ztot, s);
   mark(5);
   if (e == cudaSuccess) {
     AttnArgs a{};

@@ -17,13 +17,13 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Status-word codes written by kernels into the first bytes of the workspace.
 enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1, kDevBadIndex = 2 };
 
-// Tokens per CTA in the phi(K) / h / z pass (16 blocks).
-constexpr int kHzChunk = 1024;
+// Tokens per CTA in the phi(K) / h / z pass (8 blocks).
+constexpr int kHzChunk = 512;
 
 // Derived sizes and the byte offsets of every workspace region.
 struct Layout {
   int B, H, BH, N, Npad, Nb, d, kc, kn, nchunk;
-  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, htot32, ztot, total;
+  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, zpart, htot32, ztot, total;
 };
 
 inline Layout make_layout(const sla_params& p) {
@@ -55,6 +55,7 @@ inline Layout make_layout(const sla_params& p) {
   L.phik = take(BH * size_t(L.Npad) * d * 2);
   L.zblk = take(BH * Nb * d * 4);
   L.hpart = take(BH * size_t(L.nchunk) * d * d * 4);
+  L.zpart = take(BH * size_t(L.nchunk) * d * 4);
   L.htot32 = take(BH * d * d * 4);
   L.ztot = take(BH * d * 4);
   L.total = off;
@@ -70,8 +71,9 @@ cudaError_t launch_scores(const Layout& L, const float* qbar, const float* kbar,
 cudaError_t launch_classify(const Layout& L, const float* scores, int8_t* mc, int32_t* crit,
                             int32_t* neg, cudaStream_t s);
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
-                           __nv_bfloat16* phik, float* zblk, float* hpart, cudaStream_t s);
-cudaError_t launch_hz_reduce(const Layout& L, const float* zblk, const float* hpart, float* htot32,
+                           __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
+                           cudaStream_t s);
+cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* hpart, float* htot32,
                              float* ztot, cudaStream_t s);
 
 struct AttnArgs {
