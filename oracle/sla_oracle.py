@@ -285,15 +285,19 @@ def combine_sla2(o_s: np.ndarray, o_l: np.ndarray, alpha_h: float) -> np.ndarray
 #   * V: FP8 e4m3 per 64-token block, s_v = absmax / 448, code = e4m3(v / s_v)
 #     (round to nearest even, saturating at +-448, subnormals kept).
 #   * S = (Qc Kc^T exact integer) * s_q * s_k * softmax_scale.
-#   * P~ = exp(S - m) in (0, 1]. Each key block's V scale is folded into P
-#     relative to the largest V scale of the head, r_j = s_v,j / max_j s_v,j,
-#     and P enters the PV product as e4m3(P~ * r_j * 2^8); the row sum l uses
-#     the unquantised P~. O^s = (sum e4m3(P~ r 2^8) Vc) * max s_v / 2^8 / l.
-#   The emulation below uses the final row max m (two-pass); a kernel using a
-#   running max quantises P~ at different points, so this emulation is a
-#   diagnostic with e4m3-level agreement, not a bitwise reference.
+#   * P~ = 2^(x - m) with x = S log2(e) and m = ceil(max_j x) the row max
+#     rounded up to an integer, so P~ is in (0, 1] and its largest entry in
+#     (1/2, 1]: the FP8 scale of a row of P is a power of two. A softmax of
+#     any max offset gives the same P / l; a power-of-two scale makes the e4m3
+#     codes of P independent of which integer offset a kernel holds when it
+#     quantises (a running max only shifts the exponent).
+#   * Each key block's V scale is folded into P relative to the largest V
+#     scale of the head, r_j = s_v,j / max_j s_v,j (one float32 division), and
+#     P enters the PV product as e4m3(P~ * r_j * 2^8); the row sum l uses the
+#     unquantised P~. O^s = (sum e4m3(P~ r 2^8) Vc) * max s_v / 2^8 / l.
 
 E4M3_MAX = 448.0
+LOG2E = 1.0 / math.log(2.0)
 
 
 def e4m3_round(x: np.ndarray) -> np.ndarray:
@@ -366,8 +370,9 @@ def sparse_branch_quantized(q32: np.ndarray, k32: np.ndarray, v32: np.ndarray, M
             continue
         kblk = keys // BLOCK
         s = (qc64[r0:r1] @ kc64[keys].T) * (float(sq[i]) * sk[kblk].astype(np.float64)) * scale
-        p = np.exp(s - s.max(axis=1, keepdims=True))
-        r = sv[kblk].astype(np.float64) / sv_max
+        x = s * LOG2E
+        p = np.exp2(x - np.ceil(x.max(axis=1, keepdims=True)))
+        r = (sv[kblk] / np.float32(sv_max)).astype(np.float64)
         pq = e4m3_round(p * r[None, :] * 256.0)
         out[r0:r1] = (pq @ vq[keys]) * (sv_max / 256.0) / p.sum(axis=1, keepdims=True)
     return out

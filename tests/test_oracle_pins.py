@@ -366,9 +366,11 @@ def test_int8_block_quantisation_bounds():
 
 def test_quantized_branch_exact_when_inputs_sit_on_the_grids():
     # Q, K integer-valued with block absmax 127 (INT8 scale exactly 1), keys
-    # equal inside each block (so P~ = 1 on the critical block), V on the e4m3
-    # grid with block absmax 448 (scale 1, r_j = 1): every quantisation step is
-    # exact and the emulated branch must equal the float64 sparse branch.
+    # equal inside each block, V on the e4m3 grid with block absmax 448 (scale
+    # 1, r_j = 1): every quantisation step is exact except P's. A row's scores
+    # on its critical block are all equal to x (log2 units), so every P~ of the
+    # row is c = 2^(x - ceil x) and every P code is e4m3(256 c): the branch is
+    # the float64 sparse branch times e4m3(256 c) / (256 c), row by row.
     d, N = 8, 128
     q = RNG.integers(-20, 21, size=(N, d)).astype(np.float32)
     q[0, 0] = 127
@@ -383,7 +385,14 @@ def test_quantized_branch_exact_when_inputs_sit_on_the_grids():
     qb, kb, vb = bits(q), bits(k), bits(v)
     r = O.forward_head(qb, kb, vb, N, variant="sla2", k_crit=1, k_neg=0, alpha_h=1.0, quantized=True)
     assert (r["Mc"] == 1).sum() == 2
-    np.testing.assert_allclose(r["O_sq"], r["O_s"], rtol=1e-13, atol=1e-12)
+    crit_block = np.argmax(r["Mc"] == 1, axis=1)
+    s = np.array([q[i].astype(np.float64) @ k[64 * crit_block[i // 64]] for i in range(N)])
+    x = s / math.sqrt(d) / math.log(2.0)
+    c = 2.0 ** (x - np.ceil(x))
+    assert np.all((c > 0.5) & (c <= 1.0))
+    factor = O.e4m3_round(256.0 * c) / (256.0 * c)
+    assert np.any(factor != 1.0)  # the P step is really exercised
+    np.testing.assert_allclose(r["O_sq"], r["O_s"] * factor[:, None], rtol=1e-12, atol=1e-12)
 
 
 def test_quantized_sparse_branch_error_is_quantisation_sized():
