@@ -136,6 +136,18 @@ sla_status sla_get_mask(const sla_params* p, const void* workspace, int8_t* mc, 
 sla_status sla_get_pooled(const sla_params* p, const void* workspace, float* qbar, float* kbar,
                           void* stream);
 
+/* Quantised sparse branch (precision SLA_PREC_I8QK_F8PV): copies the codes and
+ * per-block scales of the last sla_forward() on this workspace (device to
+ * device; any output may be NULL). Source: SLA2 article (mcffsbgs.com),
+ * quantisation paragraphs (Q, K, P, V to low-bit values with scaling).
+ *   qcode, kcode  [B, H, N_pad, d] int8: clamp(rint(x / s), -127, 127), rows >= N zero.
+ *   vcode         [B, H, N_pad, d] FP8 e4m3 bytes: e4m3(v / s), RNE, saturating.
+ *   qscale, kscale [B, H, Nb] float32: absmax / 127 over the block's valid rows (1 if 0).
+ *   vscale        [B, H, Nb] float32: absmax / 448 (1 if 0).
+ * Returns SLA_ERR_INVALID_ARG for a bf16-precision parameter set. */
+sla_status sla_get_quantized(const sla_params* p, const void* workspace, int8_t* qcode, int8_t* kcode,
+                             uint8_t* vcode, float* qscale, float* kscale, float* vscale, void* stream);
+
 /* Synchronises the stream, then reads the device status word written by the
  * last sla_forward() on this workspace: SLA_OK, SLA_ERR_DEVICE_TIMEOUT if a
  * bounded in-kernel wait gave up, or SLA_ERR_DEVICE_CHECK if an in-kernel check

@@ -28,7 +28,8 @@ BLOCK = 64
 # every symbol include/sla.h declares
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate", "sla_workspace_size",
            "sla_forward", "sla_get_mask", "sla_get_pooled", "sla_read_device_status",
-           "sla_dense_forward", "sla_stage_timing", "sla_stage_times", "sla_forward_noalloc")
+           "sla_dense_forward", "sla_stage_timing", "sla_stage_times", "sla_forward_noalloc",
+           "sla_get_quantized")
 NOALLOC_WORKSPACE_BYTES = 32 << 20
 NUM_STAGES = 6
 STAGES = ("pool", "scores", "classify", "phik_hz", "hz_reduce", "attention")
@@ -77,6 +78,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sla_read_device_status": (i, [vp, vp]),
         "sla_dense_forward": (i, [vp, vp, vp, vp, i, i, i, i, ctypes.c_float, vp]),
         "sla_forward_noalloc": (i, [vp, vp, vp, vp, P, vp]),
+        "sla_get_quantized": (i, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "sla_stage_timing": (i, [i]),
         "sla_stage_times": (i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
     }
@@ -232,3 +234,21 @@ def forward_noalloc(q, k, v, *, params: Params, out=None, stream=None):
                                     _stream(stream))
     _check(st, "sla_forward_noalloc")
     return out
+
+
+def get_quantized(p: Params, workspace, stream=None):
+    """Codes and scales of the quantised sparse branch, on the device:
+    (qcode, kcode int8 [B,H,N_pad,d], vcode uint8 e4m3 bits [B,H,N_pad,d],
+    qscale, kscale, vscale float32 [B,H,Nb])."""
+    import torch
+
+    Nb = (p.N + BLOCK - 1) // BLOCK
+    dev = workspace.device
+    shp = (p.B, p.H, Nb * BLOCK, p.d)
+    qc = torch.empty(shp, dtype=torch.int8, device=dev)
+    kc = torch.empty(shp, dtype=torch.int8, device=dev)
+    vc = torch.empty(shp, dtype=torch.uint8, device=dev)
+    qs, ks, vs = (torch.empty((p.B, p.H, Nb), dtype=torch.float32, device=dev) for _ in range(3))
+    _check(load().sla_get_quantized(ctypes.byref(p), _ptr(workspace), _ptr(qc), _ptr(kc), _ptr(vc),
+                                    _ptr(qs), _ptr(ks), _ptr(vs), _stream(stream)), "sla_get_quantized")
+    return qc, kc, vc, qs, ks, vs

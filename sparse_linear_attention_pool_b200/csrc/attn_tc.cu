@@ -48,6 +48,7 @@ using namespace tc;
 
 struct TcMaps {
   CUtensorMap q, k, v, phik, w;
+  CUtensorMap qc, kc, vc;  // INT8 Q, K and e4m3 V codes (quantised sparse branch)
 };
 
 template <int D>
@@ -81,13 +82,25 @@ enum Bar {
   bKFull0, bKFull1, bKFull2, bKEmpty0, bKEmpty1, bKEmpty2,
   bVFull0, bVFull1, bVEmpty0, bVEmpty1,
   bSFull0, bSFull1, bSFree0, bSFree1, bPFull0, bPFull1, bPvDone0, bPvDone1,
-  bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, kNumBars
+  bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, bQ16Full, kNumBars
 };
 
-template <int D, int MODE>
+// QNT: the sparse branch on the quantised forms (SLA2 article, quantisation
+// paragraphs: Q, K, P, V go to low-bit values with a scale before the
+// products and are restored after). S = Qc Kc^T on kind::i8 (int32 in TMEM),
+// scaled by s_q,i s_k,j / sqrt(d); P~ = 2^(x - m) in fp32 (x = S log2 e), the
+// row sum l uses P~; P enters PV as e4m3(P~ r_j 2^4) with r_j = s_v,j / max_j
+// s_v,j (each key block's V scale folded into P); O^s = (sum P_q V_c) max s_v
+// / 2^4 / l. m is an integer running row max raised lazily: P~ <= 2^kLazy =
+// 2^4, so P~ r_j 2^4 <= 2^8 stays inside e4m3's range (448), and since m is
+// an integer the codes are the row-max-rounded-up codes e4m3(P~ r_j 2^8)
+// shifted by a power of two. The linear branch and the epilogue stay bf16
+// (phi(Q) from the bf16 Q tile).
+template <int D, int MODE, bool QNT>
 __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__ TcMaps maps,
                                                          const AttnArgs a) {
   using C = TcCfg<D>;
+  static_assert(!QNT || D == 128, "the quantised branch is built for d = 128");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -95,6 +108,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ float zs[2][D];
+  // quantised branch: per-step key-block scale and V-scale ratio, 32-step window
+  __shared__ float qwin_k[2][32], qwin_r[2][32];
+  __shared__ float qred[4];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, h = bh % a.H;
@@ -103,6 +119,11 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   const bool validB = iA + 1 < Nb;
   const int iB = validB ? iA + 1 : iA;
   constexpr bool dense = MODE == kModeDense;
+  // lazy online softmax: the running max m (log2 units) is raised only when a
+  // row's block max exceeds it by more than kLazy, so P~ <= 2^kLazy; the
+  // quantised P is P~ r_j kPMul with kPMul = 2^(8 - kLazy) <= 2^8 < 448
+  constexpr float kLazy = QNT ? 4.0f : 8.0f;
+  constexpr float kPMul = QNT ? 16.0f : 1.0f;
   const int nA = dense ? Nb : a.kc;
   const bool has_marg = !dense && (a.kc + a.kn < Nb);
   const int nE = a.kc + a.kn;
@@ -175,6 +196,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     mbar_init(bar(bOlFull), 1);
     mbar_init(bar(bYFull), 1);
     mbar_init(bar(bDrain), 1);
+    mbar_init(bar(bQ16Full), 1);
     fence_barrier_init();
   }
   if (warp == 5) tmem_alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
@@ -192,13 +214,22 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       prefetch_tmap(&maps.k);
       prefetch_tmap(&maps.v);
       if (has_marg) prefetch_tmap(&maps.phik);
-      mbar_expect_tx(bar(bQFull), 2 * C::kTile);
-      for (int s = 0; s < C::kSub; ++s) {
-        tma_load_3d(sQA + s * 8192, &maps.q, bar(bQFull), s * 64, iA * 64, bh);
-        tma_load_3d(sQB + s * 8192, &maps.q, bar(bQFull), s * 64, iB * 64, bh);
+      if constexpr (QNT) {  // INT8 Q codes: one 64 x 128-byte box per block
+        mbar_expect_tx(bar(bQFull), 2 * 8192);
+        tma_load_3d(sQA, &maps.qc, bar(bQFull), 0, iA * 64, bh);
+        tma_load_3d(sQB, &maps.qc, bar(bQFull), 0, iB * 64, bh);
+      } else {
+        mbar_expect_tx(bar(bQFull), 2 * C::kTile);
+        for (int s = 0; s < C::kSub; ++s) {
+          tma_load_3d(sQA + s * 8192, &maps.q, bar(bQFull), s * 64, iA * 64, bh);
+          tma_load_3d(sQB + s * 8192, &maps.q, bar(bQFull), s * 64, iB * 64, bh);
+        }
       }
     }
-    const int tileBytes = dense ? C::kTile : 2 * C::kTile;  // dense: one shared tile per step
+    // bytes per ring step; dense mode loads one shared tile per step, the
+    // quantised phase 1 one 8 KB code tile per block
+    const int tileBytes = dense ? C::kTile : 2 * C::kTile;
+    const int codeBytes = 2 * 8192;
     constexpr int lag = C::kNK - C::kNV;  // K copies run this many steps ahead of V copies
     int kA_reg = 0, kB_reg = 0;           // indices of the current 32-step window (K side)
     int vA_reg = 0, vB_reg = 0;           // indices of the window the V side reads
@@ -220,12 +251,18 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         const int st = TK % C::kNK;
         wait(bKEmpty0 + st, ((TK / C::kNK) & 1) ^ 1);
         if (lane == 0) {
-          const CUtensorMap* km = TK < nA ? &maps.k : &maps.phik;
           const uint32_t slot = sK + st * C::kPair;
-          mbar_expect_tx(bar(bKFull0 + st), tileBytes);
-          for (int s = 0; s < C::kSub; ++s) {
-            tma_load_3d(slot + s * 8192, km, bar(bKFull0 + st), s * 64, jA * 64, bh);
-            if (!dense) tma_load_3d(slot + C::kTile + s * 8192, km, bar(bKFull0 + st), s * 64, jB * 64, bh);
+          if (QNT && TK < nA) {
+            mbar_expect_tx(bar(bKFull0 + st), codeBytes);
+            tma_load_3d(slot, &maps.kc, bar(bKFull0 + st), 0, jA * 64, bh);
+            tma_load_3d(slot + C::kTile, &maps.kc, bar(bKFull0 + st), 0, jB * 64, bh);
+          } else {
+            const CUtensorMap* km = TK < nA ? &maps.k : &maps.phik;
+            mbar_expect_tx(bar(bKFull0 + st), tileBytes);
+            for (int s = 0; s < C::kSub; ++s) {
+              tma_load_3d(slot + s * 8192, km, bar(bKFull0 + st), s * 64, jA * 64, bh);
+              if (!dense) tma_load_3d(slot + C::kTile + s * 8192, km, bar(bKFull0 + st), s * 64, jB * 64, bh);
+            }
           }
         }
         __syncwarp();
@@ -237,13 +274,29 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         wait(bVEmpty0 + st, ((TV / C::kNV) & 1) ^ 1);
         if (lane == 0) {
           const uint32_t slot = sV + st * C::kPair;
-          mbar_expect_tx(bar(bVFull0 + st), tileBytes);
-          for (int s = 0; s < C::kSub; ++s) {
-            tma_load_3d(slot + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jA * 64, bh);
-            if (!dense) tma_load_3d(slot + C::kTile + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jB * 64, bh);
+          if (QNT && TV < nA) {
+            mbar_expect_tx(bar(bVFull0 + st), codeBytes);
+            tma_load_3d(slot, &maps.vc, bar(bVFull0 + st), 0, jA * 64, bh);
+            tma_load_3d(slot + C::kTile, &maps.vc, bar(bVFull0 + st), 0, jB * 64, bh);
+          } else {
+            mbar_expect_tx(bar(bVFull0 + st), tileBytes);
+            for (int s = 0; s < C::kSub; ++s) {
+              tma_load_3d(slot + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jA * 64, bh);
+              if (!dense) tma_load_3d(slot + C::kTile + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jB * 64, bh);
+            }
           }
         }
         __syncwarp();
+      }
+    }
+    if (lane == 0 && QNT && has_marg) {
+      // the epilogue's phi(Q) needs the bf16 Q tiles: load them over the INT8
+      // tiles once every loop product has completed
+      wait(bTailDone, 0);
+      mbar_expect_tx(bar(bQ16Full), 2 * C::kTile);
+      for (int s = 0; s < C::kSub; ++s) {
+        tma_load_3d(sQA + s * 8192, &maps.q, bar(bQ16Full), s * 64, iA * 64, bh);
+        tma_load_3d(sQB + s * 8192, &maps.q, bar(bQ16Full), s * 64, iB * 64, bh);
       }
     }
     if (use_y && lane == 0) {  // W reuses the rings once every loop product has completed
@@ -252,6 +305,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       for (int s = 0; s < C::kSub; ++s) tma_load_2d(sW + s * (D * 128), &maps.w, bar(bWFull), s * 64, 0);
       wait_drain(bWFull, 0);  // leave only after the copies have landed
     }
+    if (lane == 0 && QNT && has_marg) wait_drain(bQ16Full, 0);
   } else if (warp == 5) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
@@ -270,12 +324,25 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         tc_fence_after();
         const uint32_t vslot = sV + stv * C::kPair;
         const uint32_t pA = sP + pb * 16384, pB = pA + 8192;
+        if constexpr (QNT) {
+          // A = P e4m3 [64 rows][64 keys], 64-byte swizzled rows; B = V codes
+          // [64 tokens][128 dims] MN-major; K = 32 keys per instruction
+          constexpr uint32_t idPV8 = idesc_e4m3(64, D, 0, 1);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t acc = (tp > 0 || k > 0) ? 1u : 0u;
-          mma_bf16(tb + C::cO, sdesc(pA + k * 32, 16, 1024), sdesc(vslot + k * 2048, 8192, 1024), idPV, acc);
-          mma_bf16(tb + laneB + C::cO, sdesc(pB + k * 32, 16, 1024),
-                   sdesc(vslot + tileB + k * 2048, 8192, 1024), idPV, acc);
+          for (int k = 0; k < 2; ++k) {
+            const uint32_t acc = (tp > 0 || k > 0) ? 1u : 0u;
+            mma_e4m3(tb + C::cO, sdesc(pA + k * 32, 16, 512, 4), sdesc(vslot + k * 4096, 8192, 1024), idPV8, acc);
+            mma_e4m3(tb + laneB + C::cO, sdesc(pB + k * 32, 16, 512, 4),
+                     sdesc(vslot + C::kTile + k * 4096, 8192, 1024), idPV8, acc);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t acc = (tp > 0 || k > 0) ? 1u : 0u;
+            mma_bf16(tb + C::cO, sdesc(pA + k * 32, 16, 1024), sdesc(vslot + k * 2048, 8192, 1024), idPV, acc);
+            mma_bf16(tb + laneB + C::cO, sdesc(pB + k * 32, 16, 1024),
+                     sdesc(vslot + tileB + k * 2048, 8192, 1024), idPV, acc);
+          }
         }
         mma_commit(bar(bPvDone0 + pb));
         mma_commit(bar(bVEmpty0 + stv));
@@ -286,12 +353,23 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         wait(bSFree0 + b, ((t >> 1) & 1) ^ 1);
         tc_fence_after();
         const uint32_t kslot = sK + stk * C::kPair;
+        if constexpr (QNT) {
+          // INT8 codes, one 128-byte swizzled row per token; K = 32 per instruction
+          constexpr uint32_t idS8 = idesc_s8(64, 64);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_bf16(tb + C::cS + b * 64, sdesc(sQA + off, 16, 1024), sdesc(kslot + off, 16, 1024), idS, k > 0);
-          mma_bf16(tb + laneB + C::cS + b * 64, sdesc(sQB + off, 16, 1024),
-                   sdesc(kslot + tileB + off, 16, 1024), idS, k > 0);
+          for (int k = 0; k < D / 32; ++k) {
+            mma_s8(tb + C::cS + b * 64, sdesc(sQA + k * 32, 16, 1024), sdesc(kslot + k * 32, 16, 1024), idS8, k > 0);
+            mma_s8(tb + laneB + C::cS + b * 64, sdesc(sQB + k * 32, 16, 1024),
+                   sdesc(kslot + C::kTile + k * 32, 16, 1024), idS8, k > 0);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+            mma_bf16(tb + C::cS + b * 64, sdesc(sQA + off, 16, 1024), sdesc(kslot + off, 16, 1024), idS, k > 0);
+            mma_bf16(tb + laneB + C::cS + b * 64, sdesc(sQB + off, 16, 1024),
+                     sdesc(kslot + tileB + off, 16, 1024), idS, k > 0);
+          }
         }
         mma_commit(bar(bSFull0 + b));
         mma_commit(bar(bKEmpty0 + stk));
@@ -364,8 +442,36 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     const int jlast = dense ? Nb - 1 : checked((isB ? critB : critA)[nA - 1]);
     const bool mask_last = jlast * 64 + 64 > N;
     float m = -INFINITY, l = 0.0f;
+    // quantised branch: the row's INT8 scale and the head's largest V scale
+    float q_scale = 1.0f, sv_max = 1.0f;
+    if constexpr (QNT) {
+      const float* vs = a.vscale + size_t(bh) * Nb;
+      float vm = 0.0f;
+      for (int j = tid; j < Nb; j += 128) vm = fmaxf(vm, vs[j]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+      if (lane == 0) qred[warp] = vm;
+      named_bar(1, 128);
+      sv_max = fmaxf(fmaxf(qred[0], qred[1]), fmaxf(qred[2], qred[3]));
+      q_scale = a.qscale[size_t(bh) * Nb + blk];
+    }
 
     for (int t = 0; t < nA; ++t) {
+      if constexpr (QNT) {
+        if ((t & 31) == 0) {  // scales of the next 32 steps
+          named_bar(1, 128);
+          const int T = t + tid;
+          if (tid < 32 && T < nA) {
+#pragma unroll
+            for (int X = 0; X < 2; ++X) {
+              const int j = step_block(X, T);
+              qwin_k[X][tid] = a.kscale[size_t(bh) * Nb + j];
+              qwin_r[X][tid] = a.vscale[size_t(bh) * Nb + j] / sv_max;
+            }
+          }
+          named_bar(1, 128);
+        }
+      }
       const int b = t & 1;
       wait_w(bSFull0 + b, (t >> 1) & 1);
       tc_fence_after();
@@ -383,6 +489,14 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       }
       tc_fence_before();
       mbar_arrive(bar(bSFree0 + b));
+      // scale of this step's scores into log2 units (quantised: int32 S times
+      // s_q,i s_k,j)
+      float cs = sl2;
+      if constexpr (QNT) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) s[i] = float(__float_as_int(s[i]));
+        cs = sl2 * q_scale * qwin_k[isB][t & 31];
+      }
       if (t == nA - 1 && mask_last) {
 #pragma unroll
         for (int i = 0; i < 64; ++i)
@@ -394,16 +508,25 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 #pragma unroll
       for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * cs;
+      // quantised: m is an integer, so P~ = 2^(x - m) differs from the
+      // exact-max P~ by a power of two and its e4m3 codes are those of the
+      // exact-max P~ shifted in exponent; every rescale is an exact 2^k
       if (t == 0) {
-        m = mx;
-      } else if (__any_sync(0xffffffffu, mx > m + 8.0f)) {
-        // some row of this warp grew by more than 2^8: rescale the warp's O rows in TMEM
+        m = QNT ? ceilf(mx) : mx;
+      } else if (__any_sync(0xffffffffu, mx > m + kLazy)) {
+        // some row of this warp grew by more than 2^kLazy: rescale the warp's O rows in TMEM
         // once PV(t-1) has landed in O
         wait_w(bPvDone0 + ((t - 1) & 1), ((t - 1) >> 1) & 1);
         tc_fence_after();
-        const float mnew = fmaxf(m, mx);
-        const float corr = ex2(m - mnew);
+        const float mnew = QNT ? ceilf(fmaxf(m, mx)) : fmaxf(m, mx);
+        float corr;
+        if constexpr (QNT) {
+          const int k = int(m - mnew);  // <= 0
+          corr = k < -126 ? 0.0f : __int_as_float((k + 127) << 23);
+        } else {
+          corr = ex2(m - mnew);
+        }
         l *= corr;
         m = mnew;
 #pragma unroll
@@ -419,21 +542,33 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       }
       uint32_t pk[32];
       float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // quantised: P~ (V scale folded in) scaled by kPMul into e4m3
+      const float pq_mul = QNT ? qwin_r[isB][t & 31] * kPMul : 1.0f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2(fmaf(s[2 * i], sl2, -m));
-        const float p1 = ex2(fmaf(s[2 * i + 1], sl2, -m));
+        const float p0 = ex2(fmaf(s[2 * i], cs, -m));
+        const float p1 = ex2(fmaf(s[2 * i + 1], cs, -m));
         sum8[i & 7] += p0 + p1;
-        pk[i] = pack_bf16(p0, p1);
+        pk[i] = QNT ? pack_e4m3x2(p0 * pq_mul, p1 * pq_mul) : pack_bf16(p0, p1);
       }
       l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       // P buffer b is free once PV(t-2) has completed
       if (t >= 2) wait(bPvDone0 + b, ((t >> 1) & 1) ^ 1);
-      unsigned char* Prow = Pbase + b * 16384;
+      if constexpr (QNT) {
+        // e4m3 P row: 64 bytes, 64-byte swizzle (16-byte chunk ^= (row / 2) % 4)
+        unsigned char* Prow = Pbase - r * 128 + b * 16384 + r * 64;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(Prow + (uint32_t(c ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(Prow + (uint32_t(c ^ ((r >> 1) & 3)) << 4)) =
+              make_uint4(pk[8 * c] | (pk[8 * c + 1] << 16), pk[8 * c + 2] | (pk[8 * c + 3] << 16),
+                         pk[8 * c + 4] | (pk[8 * c + 5] << 16), pk[8 * c + 6] | (pk[8 * c + 7] << 16));
+      } else {
+        unsigned char* Prow = Pbase + b * 16384;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(Prow + (uint32_t(c ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(bar(bPFull0 + b));
@@ -441,7 +576,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     // final O: the last PV (and every earlier product) has completed
     wait_w(bPvDone0 + ((nA - 1) & 1), ((nA - 1) >> 1) & 1);
     tc_fence_after();
-    const float inv_l = 1.0f / l;
+    // quantised: undo the kPMul P scale and the V-scale fold
+    const float inv_l = (QNT ? sv_max * (1.0f / kPMul) : 1.0f) / l;
 
     float den = 1.0f;
     if (has_marg) {
@@ -478,6 +614,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         if (tid + 128 * k < 2 * D) zs[zx[k]][zc[k]] = z[k];
       // phi(Q) of this row, in place of Q (K-major swizzled tile); three passes
       // over shared memory (max, sum, write) keep the row out of registers
+      if constexpr (QNT) wait_w(bQ16Full, 0);  // bf16 Q tiles replaced the INT8 ones
       unsigned char* Qrow = smem + (isB ? C::oQB : C::oQA);
       auto qchunk = [&](int c) -> uint4* {
         return reinterpret_cast<uint4*>(Qrow + (c >> 3) * 8192 + sw128_chunk(r, c & 7));
@@ -660,13 +797,27 @@ bool map_square(CUtensorMap* m, const void* base, int D) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int MODE>
+// [BH][rows][D] one-byte codes viewed as 3D (D bytes, rows, BH); one box is a
+// 64-row x 128-byte tile (D = 128).
+bool map_codes(CUtensorMap* m, const void* base, int D, int rows, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(rows), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D), cuuint64_t(rows) * D};
+  cuuint32_t box[3] = {128, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int MODE, bool QNT = false>
 cudaError_t launch_tc(const TcMaps& maps, const AttnArgs& a, int BH, cudaStream_t s) {
   const int bytes = TcCfg<D>::kBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       bytes);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, MODE, QNT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<D, MODE><<<dim3((a.Nb + 1) / 2, BH), 192, bytes, s>>>(maps, a);
+  attn_tc_kernel<D, MODE, QNT><<<dim3((a.Nb + 1) / 2, BH), 192, bytes, s>>>(maps, a);
   return cudaGetLastError();
 }
 
@@ -680,7 +831,15 @@ cudaError_t launch_attention(const AttnArgs& a, int BH, int d, int mode, cudaStr
             map_rows(&maps.v, a.V, d, a.N, Npad, BH);
   if (ok && a.phik) ok = map_rows(&maps.phik, a.phik, d, Npad, Npad, BH);
   if (ok && a.w_proj) ok = map_square(&maps.w, a.w_proj, d);
+  const bool quant = a.qcode != nullptr;
+  if (ok && quant)
+    ok = d == 128 && mode != kModeDense && map_codes(&maps.qc, a.qcode, d, Npad, BH) &&
+         map_codes(&maps.kc, a.kcode, d, Npad, BH) && map_codes(&maps.vc, a.vcode, d, Npad, BH);
   if (!ok) return cudaErrorInvalidValue;
+  if (quant) {
+    return mode == kModeSLA ? launch_tc<128, kModeSLA, true>(maps, a, BH, s)
+                            : launch_tc<128, kModeSLA2, true>(maps, a, BH, s);
+  }
   if (d == 128) {
     if (mode == kModeSLA) return launch_tc<128, kModeSLA>(maps, a, BH, s);
     if (mode == kModeSLA2) return launch_tc<128, kModeSLA2>(maps, a, BH, s);

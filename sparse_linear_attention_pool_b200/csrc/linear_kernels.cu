@@ -29,8 +29,10 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
                                                       __nv_bfloat16* __restrict__ phik,
                                                       float* __restrict__ zblk,
                                                       float* __restrict__ hpart, float* __restrict__ zpart,
-                                                      int N, int Npad,
+                                                      uint8_t* __restrict__ vcode,
+                                                      float* __restrict__ vscale, int N, int Npad,
                                                       int Nb, int nchunk) {
+  __shared__ float vred[8];
   constexpr int CPR = D / 8;    // 16-byte chunks per row
   constexpr int WPM = 128 / D;  // warps per 16-row m tile (1 for D=128, 2 for D=64)
   constexpr int NCOL = D / WPM; // output columns per warp
@@ -129,6 +131,43 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
         *reinterpret_cast<uint32_t*>(gdst) = pk[0];
       }
     }
+    if (vcode != nullptr) {
+      // FP8 e4m3 form of V for the quantised sparse branch: scale absmax / 448
+      // over the block (s = 1 when absmax = 0), code = e4m3(v / s), round to
+      // nearest even, saturating; rows >= N are zero in the tile.
+      const __nv_bfloat16* Vt = Vs + buf * kT;
+      constexpr int kChunks = 64 * CPR / 256;  // 16-byte chunks per thread
+      float amax = 0.0f;
+#pragma unroll
+      for (int k = 0; k < kChunks; ++k) {
+        const int ch = threadIdx.x + 256 * k, r = ch / CPR, cc = ch % CPR;
+        const uint4 raw = *reinterpret_cast<const uint4*>(Vt + r * D + ((cc ^ (r & 7)) << 3));
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      if (lane == 0) vred[warp] = amax;
+      __syncthreads();
+      amax = vred[0];
+#pragma unroll
+      for (int w8 = 1; w8 < 8; ++w8) amax = fmaxf(amax, vred[w8]);
+      const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      if (threadIdx.x == 0) vscale[size_t(bh) * Nb + jb] = s;
+      uint8_t* vb = vcode + hoff + size_t(t0) * D;
+#pragma unroll
+      for (int k = 0; k < kChunks; ++k) {
+        const int ch = threadIdx.x + 256 * k, r = ch / CPR, cc = ch % CPR;
+        const uint4 raw = *reinterpret_cast<const uint4*>(Vt + r * D + ((cc ^ (r & 7)) << 3));
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t p[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          p[e >> 1] |= pack_e4m3x2(__fdiv_rn(bf16_lo(w[e]), s), __fdiv_rn(bf16_hi(w[e]), s)) << (16 * (e & 1));
+        *reinterpret_cast<uint2*>(vb + size_t(r) * D + cc * 8) = make_uint2(p[0], p[1]);
+      }
+    }
     __syncthreads();
     // H_chunk += phi(K_j)^T V_j : A = phi(K)^T (m = dim, k = token), B = V.
     // z_j = phi(K_j)^T 1 rides along as one more n-tile with B = all ones.
@@ -182,21 +221,21 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
 template <int D>
 static cudaError_t launch_hz_t(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                                __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
-                               cudaStream_t s) {
+                               uint8_t* vcode, float* vscale, cudaStream_t s) {
   const int bytes = 5 * 64 * D * 2;
   cudaError_t e =
       cudaFuncSetAttribute(phik_hz_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  phik_hz_kernel<D><<<dim3(L.nchunk, L.BH), 256, bytes, s>>>(K, V, phik, zblk, hpart, zpart, L.N, L.Npad,
-                                                            L.Nb, L.nchunk);
+  phik_hz_kernel<D><<<dim3(L.nchunk, L.BH), 256, bytes, s>>>(K, V, phik, zblk, hpart, zpart, vcode, vscale,
+                                                            L.N, L.Npad, L.Nb, L.nchunk);
   return cudaGetLastError();
 }
 
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                            __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
-                           cudaStream_t s) {
-  return L.d == 128 ? launch_hz_t<128>(L, K, V, phik, zblk, hpart, zpart, s)
-                    : launch_hz_t<64>(L, K, V, phik, zblk, hpart, zpart, s);
+                           uint8_t* vcode, float* vscale, cudaStream_t s) {
+  return L.d == 128 ? launch_hz_t<128>(L, K, V, phik, zblk, hpart, zpart, vcode, vscale, s)
+                    : launch_hz_t<64>(L, K, V, phik, zblk, hpart, zpart, vcode, vscale, s);
 }
 
 // Fixed-order sum of n strided values: 8 interleaved partial sums (element i

@@ -24,12 +24,18 @@ namespace sla {
 // ---------------------------------------------------------------------------
 // CTA: 128 threads = (128 / (d/8)) blocks x (d/8) threads; a thread owns 8
 // adjacent columns of one 64-token block. grid = (ceil(Nb / bpc), BH, 2).
+// With qcode != nullptr the same pass also writes the INT8 form of the block
+// for the quantised sparse branch: scale s = absmax / 127 over the block's
+// valid rows (s = 1 when absmax = 0), code = clamp(rint(x / s), -127, 127)
+// with x / s one rounded float32 division (rows >= N get code 0).
 template <int D>
 __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restrict__ Q,
                                                    const __nv_bfloat16* __restrict__ K,
                                                    const __nv_bfloat16* __restrict__ proj_q,
                                                    const __nv_bfloat16* __restrict__ proj_k,
                                                    float* __restrict__ qbar, float* __restrict__ kbar,
+                                                   int8_t* __restrict__ qcode, int8_t* __restrict__ kcode,
+                                                   float* __restrict__ qscale, float* __restrict__ kscale,
                                                    int N, int Npad, int Nb) {
   constexpr int TPB = D / 8;        // threads per block row
   constexpr int BPC = 128 / TPB;    // blocks per CTA
@@ -42,10 +48,13 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
   const __nv_bfloat16* X = which == 0 ? Q : K;
   const __nv_bfloat16* Wp = which == 0 ? proj_q : proj_k;
   float* out = which == 0 ? qbar : kbar;
+  int8_t* code = which == 0 ? qcode : kcode;
+  float* cscale = which == 0 ? qscale : kscale;
 
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  float amax = 0.0f;
   const bool live = blk < Nb;
   if (live) {
     const int n = min(kBlock, N - blk * kBlock);
@@ -58,8 +67,44 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
       for (int e = 0; e < 4; ++e) {
         acc[2 * e] = __fadd_rn(acc[2 * e], bf16_lo(w[e]));
         acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], bf16_hi(w[e]));
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
       }
     }
+  }
+  if (code != nullptr) {
+    // block absmax across the TPB threads of this block (contiguous lanes; all
+    // threads take part, blocks past Nb contribute 0)
+#pragma unroll
+    for (int off = TPB / 2; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (live) {
+      const int n = min(kBlock, N - blk * kBlock);
+      const __nv_bfloat16* base = X + (size_t(bh) * Npad + size_t(blk) * kBlock) * D + c0;
+      const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+      if (threadIdx.x % TPB == 0) cscale[size_t(bh) * Nb + blk] = s;
+      int8_t* cb = code + (size_t(bh) * Npad + size_t(blk) * kBlock) * D + c0;
+      for (int t = 0; t < kBlock; ++t) {
+        uint32_t lo = 0, hi = 0;
+        if (t < n) {
+          uint4 raw = *reinterpret_cast<const uint4*>(base + size_t(t) * D);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+          int q8[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            q8[2 * e] = max(-127, min(127, __float2int_rn(__fdiv_rn(bf16_lo(w[e]), s))));
+            q8[2 * e + 1] = max(-127, min(127, __float2int_rn(__fdiv_rn(bf16_hi(w[e]), s))));
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            lo |= uint32_t(q8[e] & 0xFF) << (8 * e);
+            hi |= uint32_t(q8[4 + e] & 0xFF) << (8 * e);
+          }
+        }
+        *reinterpret_cast<uint2*>(cb + size_t(t) * D) = make_uint2(lo, hi);
+      }
+    }
+  }
+  if (live) {
+    const int n = min(kBlock, N - blk * kBlock);
     if (n == kBlock) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = __fmul_rn(acc[e], 0.015625f);
@@ -98,13 +143,16 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
 
 cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                         const __nv_bfloat16* proj_q, const __nv_bfloat16* proj_k, float* qbar,
-                        float* kbar, cudaStream_t s) {
+                        float* kbar, int8_t* qcode, int8_t* kcode, float* qscale, float* kscale,
+                        cudaStream_t s) {
   const int bpc = 128 / (L.d / 8);
   dim3 grid((L.Nb + bpc - 1) / bpc, L.BH, 2);
   if (L.d == 128)
-    pool_kernel<128><<<grid, 128, 0, s>>>(Q, K, proj_q, proj_k, qbar, kbar, L.N, L.Npad, L.Nb);
+    pool_kernel<128><<<grid, 128, 0, s>>>(Q, K, proj_q, proj_k, qbar, kbar, qcode, kcode, qscale, kscale,
+                                          L.N, L.Npad, L.Nb);
   else
-    pool_kernel<64><<<grid, 128, 0, s>>>(Q, K, proj_q, proj_k, qbar, kbar, L.N, L.Npad, L.Nb);
+    pool_kernel<64><<<grid, 128, 0, s>>>(Q, K, proj_q, proj_k, qbar, kbar, qcode, kcode, qscale, kscale,
+                                         L.N, L.Npad, L.Nb);
   return cudaGetLastError();
 }
 

@@ -38,7 +38,7 @@ sla_status check_params(const sla_params* p) {
     if (p->alpha == nullptr) return SLA_ERR_INVALID_ARG;
     if ((p->proj_q == nullptr) != (p->proj_k == nullptr)) return SLA_ERR_INVALID_ARG;
   }
-  if (p->precision != SLA_PREC_BF16) return SLA_ERR_UNSUPPORTED;
+  if (p->precision == SLA_PREC_I8QK_F8PV && p->d != 128) return SLA_ERR_UNSUPPORTED;
   return SLA_OK;
 }
 
@@ -100,6 +100,12 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   float* zpart = reinterpret_cast<float*>(ws + L.zpart);
   float* htot32 = reinterpret_cast<float*>(ws + L.htot32);
   float* ztot = reinterpret_cast<float*>(ws + L.ztot);
+  int8_t* qcode = L.quant ? reinterpret_cast<int8_t*>(ws + L.qcode) : nullptr;
+  int8_t* kcode = L.quant ? reinterpret_cast<int8_t*>(ws + L.kcode) : nullptr;
+  uint8_t* vcode = L.quant ? reinterpret_cast<uint8_t*>(ws + L.vcode) : nullptr;
+  float* qscale = L.quant ? reinterpret_cast<float*>(ws + L.qscale) : nullptr;
+  float* kscale = L.quant ? reinterpret_cast<float*>(ws + L.kscale) : nullptr;
+  float* vscale = L.quant ? reinterpret_cast<float*>(ws + L.vscale) : nullptr;
   const bool sla2 = p->variant == SLA_VARIANT_SLA2;
 
   const int call = g_timer.used < g_timer.max_calls ? g_timer.used++ : -1;
@@ -110,13 +116,13 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   mark(0);
   if (e == cudaSuccess)
     e = launch_pool(L, bf(Q), bf(K), sla2 ? bf(p->proj_q) : nullptr, sla2 ? bf(p->proj_k) : nullptr,
-                    qbar, kbar, s);
+                    qbar, kbar, qcode, kcode, qscale, kscale, s);
   mark(1);
   if (e == cudaSuccess) e = launch_scores(L, qbar, kbar, scores, s);
   mark(2);
   if (e == cudaSuccess) e = launch_classify(L, scores, mc, crit, neg, s);
   mark(3);
-  if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, zpart, s);
+  if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, zpart, vcode, vscale, s);
   mark(4);
   if (e == cudaSuccess) e = launch_hz_reduce(L, zpart, hpart, htot32, ztot, s);
   mark(5);
@@ -135,6 +141,12 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
     a.w_proj = sla2 ? nullptr : bf(p->w_proj);
     a.alpha = sla2 ? p->alpha : nullptr;
     a.status = reinterpret_cast<int*>(ws + L.status);
+    a.qcode = qcode;
+    a.kcode = kcode;
+    a.vcode = vcode;
+    a.qscale = qscale;
+    a.kscale = kscale;
+    a.vscale = vscale;
     a.H = p->H;
     a.N = p->N;
     a.Nb = L.Nb;
@@ -214,6 +226,29 @@ sla_status sla_get_pooled(const sla_params* p, const void* workspace, float* qba
   if (qbar) e = cudaMemcpyAsync(qbar, ws + L.qbar, bytes, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess && kbar)
     e = cudaMemcpyAsync(kbar, ws + L.kbar, bytes, cudaMemcpyDeviceToDevice, s);
+  return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
+}
+
+sla_status sla_get_quantized(const sla_params* p, const void* workspace, int8_t* qcode, int8_t* kcode,
+                             uint8_t* vcode, float* qscale, float* kscale, float* vscale, void* stream) {
+  sla_status st = check_params(p);
+  if (st != SLA_OK) return st;
+  if (p->precision != SLA_PREC_I8QK_F8PV) return SLA_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned(workspace, 256)) return SLA_ERR_WORKSPACE;
+  const Layout L = make_layout(*p);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned char* ws = static_cast<const unsigned char*>(workspace);
+  const size_t cbytes = size_t(L.BH) * L.Npad * L.d, sbytes = size_t(L.BH) * L.Nb * 4;
+  cudaError_t e = cudaSuccess;
+  auto cp = [&](void* dst, size_t off, size_t n) {
+    if (dst && e == cudaSuccess) e = cudaMemcpyAsync(dst, ws + off, n, cudaMemcpyDeviceToDevice, s);
+  };
+  cp(qcode, L.qcode, cbytes);
+  cp(kcode, L.kcode, cbytes);
+  cp(vcode, L.vcode, cbytes);
+  cp(qscale, L.qscale, sbytes);
+  cp(kscale, L.kscale, sbytes);
+  cp(vscale, L.vscale, sbytes);
   return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
 }
 

@@ -23,7 +23,9 @@ constexpr int kHzChunk = 512;
 // Derived sizes and the byte offsets of every workspace region.
 struct Layout {
   int B, H, BH, N, Npad, Nb, d, kc, kn, nchunk;
-  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, zpart, htot32, ztot, total;
+  bool quant;  // INT8 / FP8 sparse branch: regions qcode .. vscale are present
+  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, zpart, htot32, ztot;
+  size_t qcode, kcode, vcode, qscale, kscale, vscale, total;
 };
 
 inline Layout make_layout(const sla_params& p) {
@@ -58,6 +60,15 @@ inline Layout make_layout(const sla_params& p) {
   L.zpart = take(BH * size_t(L.nchunk) * d * 4);
   L.htot32 = take(BH * d * d * 4);
   L.ztot = take(BH * d * 4);
+  L.quant = p.precision == SLA_PREC_I8QK_F8PV;
+  const size_t codes = L.quant ? BH * size_t(L.Npad) * d : 0;
+  const size_t scales = L.quant ? BH * Nb * 4 : 0;
+  L.qcode = take(codes);  // int8 [BH, Npad, d]
+  L.kcode = take(codes);  // int8 [BH, Npad, d]
+  L.vcode = take(codes);  // e4m3 [BH, Npad, d]
+  L.qscale = take(scales);
+  L.kscale = take(scales);
+  L.vscale = take(scales);
   L.total = off;
   return L;
 }
@@ -65,14 +76,15 @@ inline Layout make_layout(const sla_params& p) {
 // ---- launchers (each enqueues on `s`; returns cudaGetLastError()) ----
 cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                         const __nv_bfloat16* proj_q, const __nv_bfloat16* proj_k, float* qbar,
-                        float* kbar, cudaStream_t s);
+                        float* kbar, int8_t* qcode, int8_t* kcode, float* qscale, float* kscale,
+                        cudaStream_t s);
 cudaError_t launch_scores(const Layout& L, const float* qbar, const float* kbar, float* scores,
                           cudaStream_t s);
 cudaError_t launch_classify(const Layout& L, const float* scores, int8_t* mc, int32_t* crit,
                             int32_t* neg, cudaStream_t s);
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                            __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
-                           cudaStream_t s);
+                           uint8_t* vcode, float* vscale, cudaStream_t s);
 cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* hpart, float* htot32,
                              float* ztot, cudaStream_t s);
 
@@ -90,6 +102,13 @@ struct AttnArgs {
   const __nv_bfloat16* w_proj; // [d, d] or null
   const float* alpha;          // [H] or null
   int* status;                 // device status word (null: not reported)
+  // quantised sparse branch (null when the precision is bf16)
+  const int8_t* qcode;         // [BH, Npad, d] int8
+  const int8_t* kcode;         // [BH, Npad, d] int8
+  const uint8_t* vcode;        // [BH, Npad, d] e4m3
+  const float* qscale;         // [BH, Nb]
+  const float* kscale;         // [BH, Nb]
+  const float* vscale;         // [BH, Nb]
   int H, N, Nb, kc, kn;
   float scale_log2;            // softmax scale * log2(e)
 };
@@ -147,6 +166,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// Two floats -> packed FP8 e4m3 pair in the low 16 bits (lo in the low byte),
+// round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
+  return uint32_t(r);
 }
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }

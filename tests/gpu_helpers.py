@@ -37,15 +37,16 @@ def device_inputs(inp):
 
 
 def run_library(sla, inp, dev=None, use_w=True, use_router=True, out_fill=None, ws_fill=None):
-    """sla_forward on a workloads.Inputs. Returns dict with O (float64 numpy,
-    [B,H,N_pad,d]), Mc, crit, neg (numpy), the params and the raw tensors."""
+    """sla_forward on a workloads.Inputs, in the workload's precision. Returns
+    dict with O (float64 numpy, [B,H,N_pad,d]), Mc, crit, neg (numpy), the
+    params and the raw tensors."""
     import torch
 
     w = inp.w
     dev = dev or device_inputs(inp)
     B, H = inp.q.shape[:2]
-    p = sla.make_params(B, H, w.N, w.d, variant=w.variant, k_crit=w.k_crit, k_neg=w.k_neg,
-                        w_proj=dev["w_proj"] if use_w else None,
+    p = sla.make_params(B, H, w.N, w.d, variant=w.variant, precision=w.precision, k_crit=w.k_crit,
+                        k_neg=w.k_neg, w_proj=dev["w_proj"] if use_w else None,
                         proj_q=dev["proj_q"] if use_router else None,
                         proj_k=dev["proj_k"] if use_router else None, alpha=dev["alpha"])
     out = torch.empty_like(dev["q"])
@@ -62,8 +63,9 @@ def run_library(sla, inp, dev=None, use_w=True, use_router=True, out_fill=None, 
                 neg=neg.cpu().numpy(), params=p, ws=ws, status=st, dev=dev)
 
 
-def oracle_head(inp, idx, use_w=True, use_router=True):
-    """Oracle for entry idx (b, h) of inp.heads."""
+def oracle_head(inp, idx, use_w=True, use_router=True, quantized=False):
+    """Oracle for entry idx (b, h) of inp.heads (with quantized=True also the
+    emulated low-bit sparse branch, O_sq, and the output built from it, O_q)."""
     from oracle import sla_oracle as O
 
     w = inp.w
@@ -75,7 +77,7 @@ def oracle_head(inp, idx, use_w=True, use_router=True):
         w_proj_bits=inp.w_proj if use_w else None,
         proj_q_bits=inp.proj_q if use_router else None,
         proj_k_bits=inp.proj_k if use_router else None,
-        alpha_h=None if inp.alpha is None else float(inp.alpha[h]))
+        alpha_h=None if inp.alpha is None else float(inp.alpha[h]), quantized=quantized)
 
 
 def oracle_mask_only(inp, idx, use_router=True):
