@@ -37,6 +37,9 @@ import workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "sla_wan13b_b1h12n32768d128_s95"
 NORTH_STAR_97 = "sla2_b1h12n32768d128_s97"
+QUANT_WORKLOAD = "sla2_q_wan14b_b1h40n75600d128_s97"
+# dense tensor throughput of the 8-bit kinds relative to bf16 (2.25 vs 4.5 PFLOP/s nominal)
+LOWBIT_OVER_BF16 = 2.0
 METRIC = "ms/forward and dense-equiv TFLOPS at 95-97% sparsity; tensor-pipe % of B200 peak"
 UNIT = "TFLOPS (dense-equivalent)"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -67,6 +70,13 @@ def attention_flops(w):
     linear = BH * 2.0 * w.N * w.d * w.d
     proj = BH * 2.0 * w.N * w.d * w.d if w.variant == "sla" else 0.0
     return sparse + linear + proj
+
+
+def attention_split_flops(w):
+    """(sparse-branch FLOPs, bf16 linear/projection FLOPs) of attention_flops."""
+    BH = w.B * w.H
+    sparse = BH * w.Nb * w.k_crit * 4.0 * 64 * 64 * w.d
+    return sparse, attention_flops(w) - sparse
 
 
 def correction_flops(w):
@@ -198,9 +208,9 @@ def time_forward(sla, w, dev, steps, warmup, world, stage_timing=False, clocks=N
     """Device time of `steps` forwards (ms total, max over ranks) + per-stage ms."""
     import torch
 
-    p = sla.make_params(w.B, w.H, w.N, w.d, variant=w.variant, k_crit=w.k_crit, k_neg=w.k_neg,
-                        w_proj=dev["w_proj"], proj_q=dev["proj_q"], proj_k=dev["proj_k"],
-                        alpha=dev["alpha"])
+    p = sla.make_params(w.B, w.H, w.N, w.d, variant=w.variant, precision=w.precision,
+                        k_crit=w.k_crit, k_neg=w.k_neg, w_proj=dev["w_proj"], proj_q=dev["proj_q"],
+                        proj_k=dev["proj_k"], alpha=dev["alpha"])
     out = torch.empty_like(dev["q"])
     ws = sla.allocate_workspace(p)
     stream = torch.cuda.current_stream()
@@ -349,7 +359,8 @@ def run_ours(args):
 
     res = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "bf16" if w.precision == "bf16" else "i8/e4m3 sparse branch, bf16 linear branch",
            "data": "synthetic (seeded block-clustered Q/K, Gaussian V; Wan2.1-shaped)",
            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                       "variant": w.variant, "k_crit": w.k_crit, "k_neg": w.k_neg,
@@ -381,6 +392,25 @@ def run_ours(args):
             entry["speedup_vs_dense"] = round(res["dense_baseline"]["ms"] / ms97, 3)
         res["north_star_97"] = entry
         del dev97
+    if not args.no_quant and rank == 0 and args.workload != QUANT_WORKLOAD:
+        wq = W.WORKLOADS[QUANT_WORKLOAD]
+        devq = device_inputs(W.make_inputs(wq))
+        msq, stq, _ = time_forward(sla, wq, devq, args.steps, args.warmup, 1, stage_timing=True)
+        msq /= args.steps
+        f_lowbit, f_bf16 = attention_split_flops(wq)
+        t_attn = stq["attention"] * 1e-3
+        # time the attention kernel's products need at the measured peaks: the
+        # INT8 / e4m3 sparse products at the 8-bit rate, the rest at bf16
+        t_min = (f_lowbit / LOWBIT_OVER_BF16 + f_bf16) / (peak_tf * 1e12)
+        res["quantized"] = {
+            "workload": wq.name, "precision": wq.precision, "ms": round(msq, 4),
+            "dense_eq_tflops": round(dense_eq_flops(wq) / (msq * 1e-3) / 1e12, 2),
+            "attention_ms": round(stq["attention"], 4),
+            "attention_tflops": round((f_lowbit + f_bf16) / t_attn / 1e12, 2),
+            "attention_frac_of_mixed_peak": round(t_min / t_attn, 4),
+            "mixed_peak": f"8-bit products at {LOWBIT_OVER_BF16}x the {pk_kind} bf16 sustained peak",
+            "stages_ms": {k: round(v, 4) for k, v in stq.items()}}
+        del devq
     if not args.no_e2e:
         e_ms, h2d, d2h = time_e2e(sla, w, inp, max(3, args.steps // 4), 2, world)
         res["e2e"] = {"value": round(dense_eq_flops(w) * world / (e_ms * 1e-3) / 1e12, 3),
@@ -439,6 +469,7 @@ def main():
     ap.add_argument("--dense-steps", type=int, default=5)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-north-star", action="store_true")
+    ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

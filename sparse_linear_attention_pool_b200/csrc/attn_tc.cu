@@ -22,7 +22,8 @@
 //   warp 4     TMA producer: Q tiles, then per step the K and V tiles of both
 //              blocks (phase 1), then the phi(K) / V tiles of the excluded
 //              blocks (phase 2), then W;
-//   warp 5     MMA issuer (one thread) and TMEM owner.
+//   warp 5     MMA issuer and TMEM owner: the converged warp walks the loop,
+//              one elected lane issues each MMA and commit.
 // K tiles and V tiles travel in separate rings: a K slot is released as soon
 // as the S products that read it complete, a V slot after its PV product.
 // Phase 1 per step t: S = Q K_j^T (M=64, N=64) into one of two TMEM S
@@ -308,19 +309,21 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     if (lane == 0 && QNT && has_marg) wait_drain(bQ16Full, 0);
   } else if (warp == 5) {
     // ------------------------------ MMA issuer ------------------------------
-    if (lane == 0) {
+    // The whole warp walks the loop (warp-uniform descriptors); the MMA and
+    // commit helpers issue from one elected lane.
+    {
       constexpr uint32_t idS = idesc_bf16(64, 64, 0, 0);
       constexpr uint32_t idPV = idesc_bf16(64, D, 0, 1);
       constexpr uint32_t idG = idesc_bf16(D, D, 1, 1);
       constexpr uint32_t idN = idesc_bf16(64, D, 0, 1);
       constexpr uint32_t laneB = 16u << 16;  // block B's M=64 accumulators start at lane 16
       const uint32_t tileB = dense ? 0u : uint32_t(C::kTile);  // dense: B reads A's tile
-      wait(bQFull, 0);
+      wait_w(bQFull, 0);
       tc_fence_after();
       auto issue_pv = [&](int tp) {
         const int stv = tp % C::kNV, pb = tp & 1;
-        wait(bVFull0 + stv, (tp / C::kNV) & 1);
-        wait(bPFull0 + pb, (tp >> 1) & 1);
+        wait_w(bVFull0 + stv, (tp / C::kNV) & 1);
+        wait_w(bPFull0 + pb, (tp >> 1) & 1);
         tc_fence_after();
         const uint32_t vslot = sV + stv * C::kPair;
         const uint32_t pA = sP + pb * 16384, pB = pA + 8192;
@@ -349,8 +352,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       };
       for (int t = 0; t < nA; ++t) {
         const int stk = t % C::kNK, b = t & 1;
-        wait(bKFull0 + stk, (t / C::kNK) & 1);
-        wait(bSFree0 + b, ((t >> 1) & 1) ^ 1);
+        wait_w(bKFull0 + stk, (t / C::kNK) & 1);
+        wait_w(bSFree0 + b, ((t >> 1) & 1) ^ 1);
         tc_fence_after();
         const uint32_t kslot = sK + stk * C::kPair;
         if constexpr (QNT) {
@@ -381,8 +384,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         const uint32_t gB = D == 128 ? tb + C::cG + 128 : tb + laneB + C::cG;
         for (int u = 0; u < nE; ++u) {
           const int T = nA + u, stk = T % C::kNK, stv = T % C::kNV;
-          wait(bKFull0 + stk, (T / C::kNK) & 1);
-          wait(bVFull0 + stv, (T / C::kNV) & 1);
+          wait_w(bKFull0 + stk, (T / C::kNK) & 1);
+          wait_w(bVFull0 + stv, (T / C::kNV) & 1);
           tc_fence_after();
           const uint32_t kslot = sK + stk * C::kPair, vslot = sV + stv * C::kPair;
 #pragma unroll
@@ -398,7 +401,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       }
       mma_commit(bar(bTailDone));
       if (has_marg) {
-        wait(bHiFull, 0);
+        wait_w(bHiFull, 0);
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
@@ -410,8 +413,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         mma_commit(bar(bNumFull));
       }
       if (use_y) {
-        wait(bWFull, 0);
-        wait(bOlFull, 0);
+        wait_w(bWFull, 0);
+        wait_w(bOlFull, 0);
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
@@ -425,6 +428,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       // every MMA of this thread has completed before TMEM is released
       mma_commit(bar(bDrain));
       wait_drain(bDrain, 0);
+      __syncwarp();
     }
   } else {
     // --------------------------- softmax / epilogue ---------------------------
