@@ -43,7 +43,7 @@ LOWBIT_OVER_BF16 = 2.0
 # DRAM bytes (read + write) of one attention launch, from the ncu capture
 # summarised in profiles/attn_tc_kernel_sla_wan13b_b1h12n32768d128.md; keyed by
 # workload and valid only for the attention kernel that capture was taken of
-ATTN_TRAFFIC = {"sla_wan13b_b1h12n32768d128_s95": 419273216 + 91696128}
+ATTN_TRAFFIC = {"sla_wan13b_b1h12n32768d128_s95": 417455616 + 93460992}
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "ms/forward and dense-equiv TFLOPS at 95-97% sparsity; tensor-pipe % of B200 peak"
 UNIT = "TFLOPS (dense-equivalent)"
@@ -383,7 +383,8 @@ def run_ours(args):
            "roofline": roofline,
            "stages_ms": {k: round(v, 4) for k, v in stages.items()},
            "hbm_stages": hbm,
-           "gpu_launches": 6 * args.steps,
+           # pool, scores, classify, phi(K)/h/z, reduce, [Z_i,] attention
+           "gpu_launches": (7 if w.k_crit + w.k_neg < w.Nb else 6) * args.steps,
            "clocks": clk}
 
     if not args.no_dense and rank == 0:

@@ -20,8 +20,9 @@
 //              in TMEM lanes 0-15 of each 32-lane quarter, block B in lanes
 //              16-31: two M=64 accumulators interleaved in the same columns);
 //   warp 4     TMA producer: Q tiles, then per step the K and V tiles of both
-//              blocks (phase 1), then the phi(K) / V tiles of the excluded
-//              blocks (phase 2), then W;
+//              blocks (phase 1; bf16 at d = 128 also phi(K) into the K slot
+//              once S has read it), then the phi(K) / V tiles of the remaining
+//              excluded blocks (phase 2), then phi(Q) over the Q tiles, then W;
 //   warp 5     MMA issuer and TMEM owner: the converged warp walks the loop,
 //              one elected lane issues each MMA and commit.
 // K tiles and V tiles travel in separate rings: a K slot is released as soon
@@ -31,10 +32,12 @@
 // buffers; O += P V_j (M=64, N=d). S(t+1) is issued before PV(t), so the
 // softmax of one step overlaps the tensor-core work of the next. O is
 // rescaled in TMEM only when a row maximum grows by more than 2^8 (the
-// exponent headroom of bf16 P and fp32 O). Phase 2: G += phi(K_j)^T V_j (M=d,
-// N=d) over E_i. Epilogue: H_i = H_tot - G in bf16 -> shared memory, phi(Q_i)
-// in place of Q_i, num = phi(Q_i) H_i on the tensor core, SLA's Y = O^l W
-// likewise.
+// exponent headroom of bf16 P and fp32 O). G += phi(K_j)^T V_j (M=d, N=d) over
+// E_i: for the critical blocks right after PV(t) on the V tile already
+// resident (bf16, d = 128), for the others in phase 2. Epilogue: phi(Q_i)
+// (precomputed, loaded over Q_i) dotted with Z_i (precomputed) gives the
+// denominator; H_i = H_tot - G in bf16 -> shared memory, num = phi(Q_i) H_i on
+// the tensor core, SLA's Y = O^l W likewise.
 //
 // Every wait is bounded (about 2 s); an expired wait sets the device status
 // word to kDevTimeout and makes every later wait of the CTA return at once,
@@ -48,7 +51,7 @@ namespace sla {
 using namespace tc;
 
 struct TcMaps {
-  CUtensorMap q, k, v, phik, w;
+  CUtensorMap q, k, v, phik, w, phiq;
   CUtensorMap qc, kc, vc;  // INT8 Q, K and e4m3 V codes (quantised sparse branch)
 };
 
@@ -80,10 +83,10 @@ struct TcCfg {
 
 enum Bar {
   bQFull = 0,
-  bKFull0, bKFull1, bKFull2, bKEmpty0, bKEmpty1, bKEmpty2,
+  bKFull0, bKFull1, bKFull2, bKEmpty0, bKEmpty1, bKEmpty2, bKDone0, bKDone1, bKDone2,
   bVFull0, bVFull1, bVEmpty0, bVEmpty1,
   bSFull0, bSFull1, bSFree0, bSFree1, bPFull0, bPFull1, bPvDone0, bPvDone1,
-  bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, bQ16Full, kNumBars
+  bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, bQFree, bPhiQFull, kNumBars
 };
 
 // QNT: the sparse branch on the quantised forms (SLA2 article, quantisation
@@ -128,7 +131,17 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   const int nA = dense ? Nb : a.kc;
   const bool has_marg = !dense && (a.kc + a.kn < Nb);
   const int nE = a.kc + a.kn;
-  const int nTot = nA + (has_marg ? nE : 0);  // ring steps: phase 1 then phase 2
+  // merged mode (bf16, d = 128): the excluded-block products of the critical
+  // blocks run in phase 1 on the V tiles already resident, phi(K_j) being
+  // loaded into K_j's slot once S has read it; phase 2 then covers the
+  // negligible blocks only. The quantised branch keeps V as e4m3 codes in
+  // phase 1 and so takes every excluded block in phase 2.
+  constexpr bool kMergeCapable = !QNT && MODE != kModeDense && D == 128;
+  const bool merge = kMergeCapable && has_marg;
+  // phi(Q) and Z_i precomputed (loaded) rather than formed in the epilogue
+  const bool pre = has_marg && a.phiq != nullptr;
+  const int nP2 = has_marg ? (merge ? a.kn : nE) : 0;  // phase-2 ring steps
+  const int nTot = nA + nP2;                            // ring steps: phase 1 then phase 2
   const bool use_y = MODE == kModeSLA && a.w_proj != nullptr && has_marg;
   const int32_t* critA = a.crit + (size_t(bh) * Nb + iA) * a.kc;
   const int32_t* critB = a.crit + (size_t(bh) * Nb + iB) * a.kc;
@@ -145,13 +158,16 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     return j;
   };
   // key block of ring step T for block A (X = 0) or B (X = 1)
-  auto step_block = [&](int X, int T) {
-    if (dense) return T;
+  // u-th excluded block (the critical ones, then the negligible ones)
+  auto excl_block = [&](int X, int u) {
     const int32_t* cl = X ? critB : critA;
     const int32_t* nl = X ? negB : negA;
-    if (T < nA) return checked(cl[T]);
-    const int u = T - nA;
     return checked(u < a.kc ? cl[u] : nl[u - a.kc]);
+  };
+  auto step_block = [&](int X, int T) {
+    if (dense) return T;
+    if (T < nA) return checked((X ? critB : critA)[T]);
+    return excl_block(X, T - nA + (merge ? a.kc : 0));
   };
   auto bar = [&](int b) { return smem_u32(&bars[b]); };
   auto wait = [&](int b, uint32_t parity) { return mbar_wait(bar(b), parity, abort_flag, a.status); };
@@ -179,6 +195,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     for (int s = 0; s < C::kNK; ++s) {
       mbar_init(bar(bKFull0 + s), 1);
       mbar_init(bar(bKEmpty0 + s), 1);
+      mbar_init(bar(bKDone0 + s), 1);
     }
     for (int s = 0; s < C::kNV; ++s) {
       mbar_init(bar(bVFull0 + s), 1);
@@ -197,7 +214,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     mbar_init(bar(bOlFull), 1);
     mbar_init(bar(bYFull), 1);
     mbar_init(bar(bDrain), 1);
-    mbar_init(bar(bQ16Full), 1);
+    mbar_init(bar(bQFree), 1);
+    mbar_init(bar(bPhiQFull), 1);
     fence_barrier_init();
   }
   if (warp == 5) tmem_alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
@@ -214,7 +232,10 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       prefetch_tmap(&maps.q);
       prefetch_tmap(&maps.k);
       prefetch_tmap(&maps.v);
-      if (has_marg) prefetch_tmap(&maps.phik);
+      if (has_marg) {
+        prefetch_tmap(&maps.phik);
+        prefetch_tmap(&maps.phiq);
+      }
       if constexpr (QNT) {  // INT8 Q codes: one 64 x 128-byte box per block
         mbar_expect_tx(bar(bQFull), 2 * 8192);
         tma_load_3d(sQA, &maps.qc, bar(bQFull), 0, iA * 64, bh);
@@ -230,83 +251,156 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     // bytes per ring step; dense mode loads one shared tile per step, the
     // quantised phase 1 one 8 KB code tile per block
     const int tileBytes = dense ? C::kTile : 2 * C::kTile;
+    // phi(Q) (precomputed) over the Q or Q-code tiles once the last S product
+    // has read them: the epilogue's phi(Q) H_i and phi(Q) Z_i operand
+    auto load_phiq = [&]() {
+      wait(bQFree, 0);
+      if (lane == 0) {
+        mbar_expect_tx(bar(bPhiQFull), 2 * C::kTile);
+        for (int s = 0; s < C::kSub; ++s) {
+          tma_load_3d(sQA + s * 8192, &maps.phiq, bar(bPhiQFull), s * 64, iA * 64, bh);
+          tma_load_3d(sQB + s * 8192, &maps.phiq, bar(bPhiQFull), s * 64, iB * 64, bh);
+        }
+      }
+      __syncwarp();
+    };
     const int codeBytes = 2 * 8192;
     constexpr int lag = C::kNK - C::kNV;  // K copies run this many steps ahead of V copies
     int kA_reg = 0, kB_reg = 0;           // indices of the current 32-step window (K side)
     int vA_reg = 0, vB_reg = 0;           // indices of the window the V side reads
-    for (int T = 0; T < nTot + lag; ++T) {
-      const int TK = T, TV = T - lag;
-      if ((TK & 31) == 0 && TK < nTot) {
-        const int Ti = TK + lane;
-        kA_reg = Ti < nTot ? step_block(0, Ti) : 0;
-        kB_reg = Ti < nTot ? step_block(1, Ti) : 0;
-      }
-      if (TV >= 0 && (TV & 31) == 0 && TV < nTot) {
-        const int Ti = TV + lane;
-        vA_reg = Ti < nTot ? step_block(0, Ti) : 0;
-        vB_reg = Ti < nTot ? step_block(1, Ti) : 0;
-      }
-      if (TK < nTot) {
-        const int jA = __shfl_sync(0xffffffffu, kA_reg, TK & 31);
-        const int jB = __shfl_sync(0xffffffffu, kB_reg, TK & 31);
-        const int st = TK % C::kNK;
-        wait(bKEmpty0 + st, ((TK / C::kNK) & 1) ^ 1);
-        if (lane == 0) {
-          const uint32_t slot = sK + st * C::kPair;
-          if (QNT && TK < nA) {
-            mbar_expect_tx(bar(bKFull0 + st), codeBytes);
-            tma_load_3d(slot, &maps.kc, bar(bKFull0 + st), 0, jA * 64, bh);
-            tma_load_3d(slot + C::kTile, &maps.kc, bar(bKFull0 + st), 0, jB * 64, bh);
-          } else {
-            const CUtensorMap* km = TK < nA ? &maps.k : &maps.phik;
-            mbar_expect_tx(bar(bKFull0 + st), tileBytes);
-            for (int s = 0; s < C::kSub; ++s) {
-              tma_load_3d(slot + s * 8192, km, bar(bKFull0 + st), s * 64, jA * 64, bh);
-              if (!dense) tma_load_3d(slot + C::kTile + s * 8192, km, bar(bKFull0 + st), s * 64, jB * 64, bh);
+    if (!merge) {
+      for (int T = 0; T < nTot + lag; ++T) {
+        const int TK = T, TV = T - lag;
+        if ((TK & 31) == 0 && TK < nTot) {
+          const int Ti = TK + lane;
+          kA_reg = Ti < nTot ? step_block(0, Ti) : 0;
+          kB_reg = Ti < nTot ? step_block(1, Ti) : 0;
+        }
+        if (TV >= 0 && (TV & 31) == 0 && TV < nTot) {
+          const int Ti = TV + lane;
+          vA_reg = Ti < nTot ? step_block(0, Ti) : 0;
+          vB_reg = Ti < nTot ? step_block(1, Ti) : 0;
+        }
+        if (TK < nTot) {
+          const int jA = __shfl_sync(0xffffffffu, kA_reg, TK & 31);
+          const int jB = __shfl_sync(0xffffffffu, kB_reg, TK & 31);
+          const int st = TK % C::kNK;
+          wait(bKEmpty0 + st, ((TK / C::kNK) & 1) ^ 1);
+          if (lane == 0) {
+            const uint32_t slot = sK + st * C::kPair;
+            if (QNT && TK < nA) {
+              mbar_expect_tx(bar(bKFull0 + st), codeBytes);
+              tma_load_3d(slot, &maps.kc, bar(bKFull0 + st), 0, jA * 64, bh);
+              tma_load_3d(slot + C::kTile, &maps.kc, bar(bKFull0 + st), 0, jB * 64, bh);
+            } else {
+              const CUtensorMap* km = TK < nA ? &maps.k : &maps.phik;
+              mbar_expect_tx(bar(bKFull0 + st), tileBytes);
+              for (int s = 0; s < C::kSub; ++s) {
+                tma_load_3d(slot + s * 8192, km, bar(bKFull0 + st), s * 64, jA * 64, bh);
+                if (!dense) tma_load_3d(slot + C::kTile + s * 8192, km, bar(bKFull0 + st), s * 64, jB * 64, bh);
+              }
             }
           }
+          __syncwarp();
         }
+        if (TV >= 0 && TV < nTot) {
+          const int jA = __shfl_sync(0xffffffffu, vA_reg, TV & 31);
+          const int jB = __shfl_sync(0xffffffffu, vB_reg, TV & 31);
+          const int st = TV % C::kNV;
+          wait(bVEmpty0 + st, ((TV / C::kNV) & 1) ^ 1);
+          if (lane == 0) {
+            const uint32_t slot = sV + st * C::kPair;
+            if (QNT && TV < nA) {
+              mbar_expect_tx(bar(bVFull0 + st), codeBytes);
+              tma_load_3d(slot, &maps.vc, bar(bVFull0 + st), 0, jA * 64, bh);
+              tma_load_3d(slot + C::kTile, &maps.vc, bar(bVFull0 + st), 0, jB * 64, bh);
+            } else {
+              mbar_expect_tx(bar(bVFull0 + st), tileBytes);
+              for (int s = 0; s < C::kSub; ++s) {
+                tma_load_3d(slot + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jA * 64, bh);
+                if (!dense) tma_load_3d(slot + C::kTile + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jB * 64, bh);
+              }
+            }
+          }
+          __syncwarp();
+        }
+      }
+    } else {
+      // Merged mode. Step t: K(t); then, one step behind, V(t-1) and phi(K)(t-1)
+      // into K(t-1)'s slot once S(t-1) has read it (KDone). Phase 2: phi(K) and
+      // V of the negligible blocks. A K slot is filled twice per phase-1 step,
+      // so its barrier phases are tracked per slot in bit masks.
+      auto load_pair = [&](uint32_t slot, const CUtensorMap* m, uint32_t fb, int jA, int jB) {
+        mbar_expect_tx(fb, 2 * C::kTile);
+        for (int s = 0; s < C::kSub; ++s) {
+          tma_load_3d(slot + s * 8192, m, fb, s * 64, jA * 64, bh);
+          tma_load_3d(slot + C::kTile + s * 8192, m, fb, s * 64, jB * 64, bh);
+        }
+      };
+      uint32_t pe = (1u << C::kNK) - 1;  // KEmpty parity per slot (a slot's first fill passes)
+      uint32_t pd = 0;                   // KDone parity per slot
+      for (int t = 0; t <= nA; ++t) {
+        if ((t & 31) == 0 && t < nA) {
+          const int Ti = t + lane;
+          kA_reg = Ti < nA ? step_block(0, Ti) : 0;
+          kB_reg = Ti < nA ? step_block(1, Ti) : 0;
+        }
+        if (t >= 1 && ((t - 1) & 31) == 0) {
+          const int Ti = t - 1 + lane;
+          vA_reg = Ti < nA ? step_block(0, Ti) : 0;
+          vB_reg = Ti < nA ? step_block(1, Ti) : 0;
+        }
+        if (t < nA) {  // K(t)
+          const int jA = __shfl_sync(0xffffffffu, kA_reg, t & 31);
+          const int jB = __shfl_sync(0xffffffffu, kB_reg, t & 31);
+          const int st = t % C::kNK;
+          wait(bKEmpty0 + st, (pe >> st) & 1u);
+          pe ^= 1u << st;
+          if (lane == 0) load_pair(sK + st * C::kPair, &maps.k, bar(bKFull0 + st), jA, jB);
+          __syncwarp();
+        }
+        if (t >= 1) {  // V(t-1), then phi(K)(t-1)
+          const int u = t - 1;
+          const int jA = __shfl_sync(0xffffffffu, vA_reg, u & 31);
+          const int jB = __shfl_sync(0xffffffffu, vB_reg, u & 31);
+          const int sv = u % C::kNV, st = u % C::kNK;
+          wait(bVEmpty0 + sv, ((u / C::kNV) & 1) ^ 1);
+          if (lane == 0) load_pair(sV + sv * C::kPair, &maps.v, bar(bVFull0 + sv), jA, jB);
+          __syncwarp();
+          wait(bKDone0 + st, (pd >> st) & 1u);
+          pd ^= 1u << st;
+          if (lane == 0) load_pair(sK + st * C::kPair, &maps.phik, bar(bKFull0 + st), jA, jB);
+          __syncwarp();
+        }
+      }
+      if (pre) load_phiq();  // S(nA-1) has completed: phi(K)(nA-1) waited for it
+      for (int u = 0; u < nP2; ++u) {  // the negligible blocks
+        const int T = nA + u;
+        if ((u & 31) == 0) {
+          const int Ti = T + lane;
+          kA_reg = Ti < nTot ? step_block(0, Ti) : 0;
+          kB_reg = Ti < nTot ? step_block(1, Ti) : 0;
+        }
+        const int jA = __shfl_sync(0xffffffffu, kA_reg, u & 31);
+        const int jB = __shfl_sync(0xffffffffu, kB_reg, u & 31);
+        const int st = T % C::kNK, sv = T % C::kNV;
+        wait(bKEmpty0 + st, (pe >> st) & 1u);
+        pe ^= 1u << st;
+        if (lane == 0) load_pair(sK + st * C::kPair, &maps.phik, bar(bKFull0 + st), jA, jB);
         __syncwarp();
-      }
-      if (TV >= 0 && TV < nTot) {
-        const int jA = __shfl_sync(0xffffffffu, vA_reg, TV & 31);
-        const int jB = __shfl_sync(0xffffffffu, vB_reg, TV & 31);
-        const int st = TV % C::kNV;
-        wait(bVEmpty0 + st, ((TV / C::kNV) & 1) ^ 1);
-        if (lane == 0) {
-          const uint32_t slot = sV + st * C::kPair;
-          if (QNT && TV < nA) {
-            mbar_expect_tx(bar(bVFull0 + st), codeBytes);
-            tma_load_3d(slot, &maps.vc, bar(bVFull0 + st), 0, jA * 64, bh);
-            tma_load_3d(slot + C::kTile, &maps.vc, bar(bVFull0 + st), 0, jB * 64, bh);
-          } else {
-            mbar_expect_tx(bar(bVFull0 + st), tileBytes);
-            for (int s = 0; s < C::kSub; ++s) {
-              tma_load_3d(slot + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jA * 64, bh);
-              if (!dense) tma_load_3d(slot + C::kTile + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jB * 64, bh);
-            }
-          }
-        }
+        wait(bVEmpty0 + sv, ((T / C::kNV) & 1) ^ 1);
+        if (lane == 0) load_pair(sV + sv * C::kPair, &maps.v, bar(bVFull0 + sv), jA, jB);
         __syncwarp();
       }
     }
-    if (lane == 0 && QNT && has_marg) {
-      // the epilogue's phi(Q) needs the bf16 Q tiles: load them over the INT8
-      // tiles once every loop product has completed
-      wait(bTailDone, 0);
-      mbar_expect_tx(bar(bQ16Full), 2 * C::kTile);
-      for (int s = 0; s < C::kSub; ++s) {
-        tma_load_3d(sQA + s * 8192, &maps.q, bar(bQ16Full), s * 64, iA * 64, bh);
-        tma_load_3d(sQB + s * 8192, &maps.q, bar(bQ16Full), s * 64, iB * 64, bh);
-      }
-    }
+    if (pre && !merge) load_phiq();
     if (use_y && lane == 0) {  // W reuses the rings once every loop product has completed
       wait(bTailDone, 0);
       mbar_expect_tx(bar(bWFull), C::kMat);
       for (int s = 0; s < C::kSub; ++s) tma_load_2d(sW + s * (D * 128), &maps.w, bar(bWFull), s * 64, 0);
       wait_drain(bWFull, 0);  // leave only after the copies have landed
     }
-    if (lane == 0 && QNT && has_marg) wait_drain(bQ16Full, 0);
+    if (lane == 0 && pre) wait_drain(bPhiQFull, 0);
   } else if (warp == 5) {
     // ------------------------------ MMA issuer ------------------------------
     // The whole warp walks the loop (warp-uniform descriptors); the MMA and
@@ -348,11 +442,37 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           }
         }
         mma_commit(bar(bPvDone0 + pb));
+        if (!merge) mma_commit(bar(bVEmpty0 + stv));  // merged: released after G
+      };
+      const uint32_t gA = tb + C::cG;
+      const uint32_t gB = D == 128 ? tb + C::cG + 128 : tb + laneB + C::cG;
+      // G += phi(K_j)^T V_j for both blocks (M = N = D, MN-major operands)
+      auto issue_g = [&](uint32_t kslot, uint32_t vslot, bool first) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = (!first || k > 0) ? 1u : 0u;
+          mma_bf16(gA, sdesc(kslot + k * 2048, 8192, 1024), sdesc(vslot + k * 2048, 8192, 1024), idG, acc);
+          mma_bf16(gB, sdesc(kslot + C::kTile + k * 2048, 8192, 1024),
+                   sdesc(vslot + C::kTile + k * 2048, 8192, 1024), idG, acc);
+        }
+      };
+      uint32_t kf = 0;  // KFull parity per slot
+      auto wait_kfull = [&](int stk) {
+        wait_w(bKFull0 + stk, (kf >> stk) & 1u);
+        kf ^= 1u << stk;
+      };
+      // merged mode: G for critical step tp, after PV(tp), on phi(K)(tp) and V(tp)
+      auto issue_g1 = [&](int tp) {
+        const int stk = tp % C::kNK, stv = tp % C::kNV;
+        wait_kfull(stk);
+        tc_fence_after();
+        issue_g(sK + stk * C::kPair, sV + stv * C::kPair, tp == 0);
+        mma_commit(bar(bKEmpty0 + stk));
         mma_commit(bar(bVEmpty0 + stv));
       };
       for (int t = 0; t < nA; ++t) {
         const int stk = t % C::kNK, b = t & 1;
-        wait_w(bKFull0 + stk, (t / C::kNK) & 1);
+        wait_kfull(stk);
         wait_w(bSFree0 + b, ((t >> 1) & 1) ^ 1);
         tc_fence_after();
         const uint32_t kslot = sK + stk * C::kPair;
@@ -375,29 +495,25 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           }
         }
         mma_commit(bar(bSFull0 + b));
-        mma_commit(bar(bKEmpty0 + stk));
-        if (t > 0) issue_pv(t - 1);
-      }
-      if (nA > 0) issue_pv(nA - 1);
-      if (has_marg) {
-        const uint32_t gA = tb + C::cG;
-        const uint32_t gB = D == 128 ? tb + C::cG + 128 : tb + laneB + C::cG;
-        for (int u = 0; u < nE; ++u) {
-          const int T = nA + u, stk = T % C::kNK, stv = T % C::kNV;
-          wait_w(bKFull0 + stk, (T / C::kNK) & 1);
-          wait_w(bVFull0 + stv, (T / C::kNV) & 1);
-          tc_fence_after();
-          const uint32_t kslot = sK + stk * C::kPair, vslot = sV + stv * C::kPair;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t acc = (u > 0 || k > 0) ? 1u : 0u;
-            mma_bf16(gA, sdesc(kslot + k * 2048, 8192, 1024), sdesc(vslot + k * 2048, 8192, 1024), idG, acc);
-            mma_bf16(gB, sdesc(kslot + C::kTile + k * 2048, 8192, 1024),
-                     sdesc(vslot + C::kTile + k * 2048, 8192, 1024), idG, acc);
-          }
-          mma_commit(bar(bKEmpty0 + stk));
-          mma_commit(bar(bVEmpty0 + stv));
+        mma_commit(bar(merge ? bKDone0 + stk : bKEmpty0 + stk));  // merged: phi(K) refills the slot
+        if (pre && t == nA - 1) mma_commit(bar(bQFree));          // Q tiles free for phi(Q)
+        if (t > 0) {
+          issue_pv(t - 1);
+          if (merge) issue_g1(t - 1);
         }
+      }
+      if (nA > 0) {
+        issue_pv(nA - 1);
+        if (merge) issue_g1(nA - 1);
+      }
+      for (int u = 0; u < nP2; ++u) {  // phase 2
+        const int T = nA + u, stk = T % C::kNK, stv = T % C::kNV;
+        wait_kfull(stk);
+        wait_w(bVFull0 + stv, (T / C::kNV) & 1);
+        tc_fence_after();
+        issue_g(sK + stk * C::kPair, sV + stv * C::kPair, !merge && u == 0);
+        mma_commit(bar(bKEmpty0 + stk));
+        mma_commit(bar(bVEmpty0 + stv));
       }
       mma_commit(bar(bTailDone));
       if (has_marg) {
@@ -584,7 +700,29 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     const float inv_l = (QNT ? sv_max * (1.0f / kPMul) : 1.0f) / l;
 
     float den = 1.0f;
-    if (has_marg) {
+    if (pre) {
+      // Z_i of blocks A and B (precomputed), then den = phi(Q_i) . Z_i from the
+      // phi(Q) tile the producer loads over Q once the last S product is done
+      const float* zia = a.zi + (size_t(bh) * Nb + iA) * D;
+      const float* zib = a.zi + (size_t(bh) * Nb + iB) * D;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = tid + 128 * k;
+        if (e < 2 * D) zs[e / D][e % D] = (e < D ? zia : zib)[e % D];
+      }
+      named_bar(1, 128);  // zs complete
+      wait_w(bPhiQFull, 0);
+      const unsigned char* Qrow = smem + (isB ? C::oQB : C::oQA);
+      den = 0.0f;
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(Qrow + (c >> 3) * 8192 + sw128_chunk(r, c & 7));
+        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          den += bf16_lo(wv[e]) * zs[isB][8 * c + 2 * e] + bf16_hi(wv[e]) * zs[isB][8 * c + 2 * e + 1];
+      }
+    } else if (has_marg) {
       // Z_i = Z_tot - sum over the excluded blocks of z_j, blocks A and B.
       // Thread handles (X, c) for e = tid and tid + 128 < 2D; block indices are
       // fetched 32 at a time, one per lane, and broadcast.
@@ -601,8 +739,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       }
       for (int u0 = 0; u0 < nE; u0 += 32) {
         const int uu = u0 + lane;
-        const int myA = uu < nE ? step_block(0, nA + uu) : 0;
-        const int myB = uu < nE ? step_block(1, nA + uu) : 0;
+        const int myA = uu < nE ? excl_block(0, uu) : 0;
+        const int myB = uu < nE ? excl_block(1, uu) : 0;
         const int cnt = min(32, nE - u0);
 #pragma unroll 4
         for (int i = 0; i < cnt; ++i) {
@@ -616,9 +754,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 #pragma unroll
       for (int k = 0; k < 2; ++k)
         if (tid + 128 * k < 2 * D) zs[zx[k]][zc[k]] = z[k];
-      // phi(Q) of this row, in place of Q (K-major swizzled tile); three passes
-      // over shared memory (max, sum, write) keep the row out of registers
-      if constexpr (QNT) wait_w(bQ16Full, 0);  // bf16 Q tiles replaced the INT8 ones
+      // phi(Q) of this row, in place of the bf16 Q tile (K-major swizzled);
+      // three passes over shared memory (max, sum, write) keep the row out of
+      // registers
       unsigned char* Qrow = smem + (isB ? C::oQB : C::oQA);
       auto qchunk = [&](int c) -> uint4* {
         return reinterpret_cast<uint4*>(Qrow + (c >> 3) * 8192 + sw128_chunk(r, c & 7));
@@ -654,6 +792,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         }
         *qchunk(c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
+    }
+    if (has_marg) {
       // H_i = H_tot - G_i -> bf16, MN-major tile [D rows c][D cols e]
       wait_w(bTailDone, 0);
       tc_fence_after();
@@ -834,8 +974,11 @@ cudaError_t launch_attention(const AttnArgs& a, int BH, int d, int mode, cudaStr
   bool ok = map_rows(&maps.q, a.Q, d, a.N, Npad, BH) && map_rows(&maps.k, a.K, d, a.N, Npad, BH) &&
             map_rows(&maps.v, a.V, d, a.N, Npad, BH);
   if (ok && a.phik) ok = map_rows(&maps.phik, a.phik, d, Npad, Npad, BH);
+  if (ok && a.phiq) ok = map_rows(&maps.phiq, a.phiq, d, a.N, Npad, BH);
   if (ok && a.w_proj) ok = map_square(&maps.w, a.w_proj, d);
   const bool quant = a.qcode != nullptr;
+  // the quantised branch's Q tiles hold INT8 codes: its phi(Q) must come precomputed
+  if (quant && a.kc + a.kn < a.Nb && a.phiq == nullptr) return cudaErrorInvalidValue;
   if (ok && quant)
     ok = d == 128 && mode != kModeDense && map_codes(&maps.qc, a.qcode, d, Npad, BH) &&
          map_codes(&maps.kc, a.kcode, d, Npad, BH) && map_codes(&maps.vc, a.vcode, d, Npad, BH);

@@ -278,4 +278,58 @@ cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* h
   return cudaGetLastError();
 }
 
+// Z_i = Z_tot - sum over the excluded blocks of query block i (its critical
+// blocks, then its negligible ones, in list order) of z_j: the denominator
+// vector of the linear branch ([SLA-sum] formula 3, the sum over the marginal
+// blocks formed as a complement). One warp per query block, d / 32 columns per
+// lane. A list entry outside [0, Nb) is clamped and flagged in the status word.
+__global__ void __launch_bounds__(256) zi_kernel(const int32_t* __restrict__ crit,
+                                                 const int32_t* __restrict__ neg,
+                                                 const float* __restrict__ zblk,
+                                                 const float* __restrict__ ztot, float* __restrict__ zi,
+                                                 int* status, int Nb, int kc, int kn, int d) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + warp, bh = blockIdx.y;
+  if (i >= Nb) return;
+  const int32_t* cl = crit + (size_t(bh) * Nb + i) * kc;
+  const int32_t* nl = neg + (size_t(bh) * Nb + i) * (kn > 0 ? kn : 1);
+  const float* zb = zblk + size_t(bh) * Nb * d;
+  const int per = d / 32;
+  float z[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) z[q] = q < per ? ztot[size_t(bh) * d + lane + 32 * q] : 0.0f;
+  const int ne = kc + kn;
+  // list entries 32 at a time (one per lane, broadcast), so the row loads of a
+  // batch are independent of each other
+  for (int u0 = 0; u0 < ne; u0 += 32) {
+    const int u = u0 + lane;
+    int my = 0;
+    if (u < ne) {
+      my = u < kc ? cl[u] : nl[u - kc];
+      if (my < 0 || my >= Nb) {
+        if (status != nullptr) atomicExch(status, kDevBadIndex);
+        my = my < 0 ? 0 : Nb - 1;
+      }
+    }
+    const int cnt = min(32, ne - u0);
+#pragma unroll 8
+    for (int k = 0; k < cnt; ++k) {
+      const int j = __shfl_sync(0xffffffffu, my, k);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q < per) z[q] -= zb[size_t(j) * d + lane + 32 * q];
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (q < per) zi[(size_t(bh) * Nb + i) * d + lane + 32 * q] = z[q];
+}
+
+cudaError_t launch_zi(const Layout& L, const int32_t* crit, const int32_t* neg, const float* zblk,
+                      const float* ztot, float* zi, int* status, cudaStream_t s) {
+  dim3 grid((L.Nb + 7) / 8, L.BH);
+  zi_kernel<<<grid, 256, 0, s>>>(crit, neg, zblk, ztot, zi, status, L.Nb, L.kc, L.kn, L.d);
+  return cudaGetLastError();
+}
+
 }  // namespace sla

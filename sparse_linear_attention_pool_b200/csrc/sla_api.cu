@@ -100,6 +100,8 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   float* zpart = reinterpret_cast<float*>(ws + L.zpart);
   float* htot32 = reinterpret_cast<float*>(ws + L.htot32);
   float* ztot = reinterpret_cast<float*>(ws + L.ztot);
+  __nv_bfloat16* phiq = L.pre ? reinterpret_cast<__nv_bfloat16*>(ws + L.phiq) : nullptr;
+  float* zi = L.pre ? reinterpret_cast<float*>(ws + L.zi) : nullptr;
   int8_t* qcode = L.quant ? reinterpret_cast<int8_t*>(ws + L.qcode) : nullptr;
   int8_t* kcode = L.quant ? reinterpret_cast<int8_t*>(ws + L.kcode) : nullptr;
   uint8_t* vcode = L.quant ? reinterpret_cast<uint8_t*>(ws + L.vcode) : nullptr;
@@ -116,7 +118,7 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   mark(0);
   if (e == cudaSuccess)
     e = launch_pool(L, bf(Q), bf(K), sla2 ? bf(p->proj_q) : nullptr, sla2 ? bf(p->proj_k) : nullptr,
-                    qbar, kbar, qcode, kcode, qscale, kscale, s);
+                    qbar, kbar, qcode, kcode, qscale, kscale, phiq, s);
   mark(1);
   if (e == cudaSuccess) e = launch_scores(L, qbar, kbar, scores, s);
   mark(2);
@@ -125,6 +127,8 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, zpart, vcode, vscale, s);
   mark(4);
   if (e == cudaSuccess) e = launch_hz_reduce(L, zpart, hpart, htot32, ztot, s);
+  if (e == cudaSuccess && L.pre)
+    e = launch_zi(L, crit, neg, zblk, ztot, zi, reinterpret_cast<int*>(ws + L.status), s);
   mark(5);
   if (e == cudaSuccess) {
     AttnArgs a{};
@@ -136,6 +140,8 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
     a.crit = crit;
     a.neg = neg;
     a.htot32 = htot32;
+    a.phiq = phiq;
+    a.zi = zi;
     a.ztot = ztot;
     a.zblk = zblk;
     a.w_proj = sla2 ? nullptr : bf(p->w_proj);

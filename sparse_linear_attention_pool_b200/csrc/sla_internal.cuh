@@ -24,7 +24,10 @@ constexpr int kHzChunk = 512;
 struct Layout {
   int B, H, BH, N, Npad, Nb, d, kc, kn, nchunk;
   bool quant;  // INT8 / FP8 sparse branch: regions qcode .. vscale are present
-  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, zpart, htot32, ztot;
+  bool linear;  // a marginal block exists (the linear branch is computed)
+  bool pre;     // phi(Q) and Z_i are precomputed (regions phiq, zi) instead of
+                // formed inside the attention kernel
+  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, zpart, htot32, ztot, phiq, zi;
   size_t qcode, kcode, vcode, qscale, kscale, vscale, total;
 };
 
@@ -60,6 +63,16 @@ inline Layout make_layout(const sla_params& p) {
   L.zpart = take(BH * size_t(L.nchunk) * d * 4);
   L.htot32 = take(BH * d * d * 4);
   L.ztot = take(BH * d * 4);
+  L.linear = L.kc + L.kn < L.Nb;
+  // The attention kernel forms Z_i (about 350 cycles per excluded block) and
+  // phi(Q) (about 8000 cycles) itself while the excluded-block products of
+  // phase 2 stream (about 1260 cycles per negligible block at d = 128); when
+  // phase 2 is too short to hide that, both are precomputed instead. The
+  // quantised branch always precomputes: its Q tiles hold INT8 codes.
+  L.pre = L.linear && (p.precision == SLA_PREC_I8QK_F8PV ||
+                       size_t(L.kn) * 1260 < size_t(L.kc + L.kn) * 350 + 8000);
+  L.phiq = take(L.pre ? BH * size_t(L.Npad) * d * 2 : 0);  // phi(Q) bf16 [BH, Npad, d]
+  L.zi = take(L.pre ? BH * Nb * d * 4 : 0);               // Z_i fp32 [BH, Nb, d]
   L.quant = p.precision == SLA_PREC_I8QK_F8PV;
   const size_t codes = L.quant ? BH * size_t(L.Npad) * d : 0;
   const size_t scales = L.quant ? BH * Nb * 4 : 0;
@@ -77,7 +90,7 @@ inline Layout make_layout(const sla_params& p) {
 cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                         const __nv_bfloat16* proj_q, const __nv_bfloat16* proj_k, float* qbar,
                         float* kbar, int8_t* qcode, int8_t* kcode, float* qscale, float* kscale,
-                        cudaStream_t s);
+                        __nv_bfloat16* phiq, cudaStream_t s);
 cudaError_t launch_scores(const Layout& L, const float* qbar, const float* kbar, float* scores,
                           cudaStream_t s);
 cudaError_t launch_classify(const Layout& L, const float* scores, int8_t* mc, int32_t* crit,
@@ -87,6 +100,9 @@ cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_b
                            uint8_t* vcode, float* vscale, cudaStream_t s);
 cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* hpart, float* htot32,
                              float* ztot, cudaStream_t s);
+// Z_i = Z_tot - sum of z_j over the excluded blocks of query block i
+cudaError_t launch_zi(const Layout& L, const int32_t* crit, const int32_t* neg, const float* zblk,
+                      const float* ztot, float* zi, int* status, cudaStream_t s);
 
 struct AttnArgs {
   const __nv_bfloat16* Q;
@@ -97,8 +113,10 @@ struct AttnArgs {
   const int32_t* crit;         // [BH, Nb, kc]
   const int32_t* neg;          // [BH, Nb, kn]
   const float* htot32;         // [BH, d, d]  H_tot = sum_j phi(K_j)^T V_j
-  const float* ztot;           // [BH, d]     Z_tot = sum_j z_j
-  const float* zblk;           // [BH, Nb, d] z_j
+  const __nv_bfloat16* phiq;   // [BH, Npad, d] phi(Q), or null: formed in the kernel
+  const float* zi;             // [BH, Nb, d] Z_i, or null: formed in the kernel
+  const float* ztot;           // [BH, d] Z_tot (in-kernel Z_i)
+  const float* zblk;           // [BH, Nb, d] z_j (in-kernel Z_i)
   const __nv_bfloat16* w_proj; // [d, d] or null
   const float* alpha;          // [H] or null
   int* status;                 // device status word (null: not reported)
@@ -173,6 +191,13 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
   return uint32_t(r);
+}
+constexpr float kLog2e = 1.4426950408889634f;
+// 2^x on the MUFU unit (approximate, flushes subnormals)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }

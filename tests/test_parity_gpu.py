@@ -55,6 +55,13 @@ EDGE = [
     ("no_router", 1, 1, 64 * 9 + 33, 128, "sla2", 3, 0, True, False),
     ("batch2_heads3", 2, 3, 64 * 11 + 5, 128, "sla", 3, 2, True, True),
     ("many_blocks_d64", 1, 1, 64 * 40, 64, "sla", 4, 8, True, True),
+    # Z_i and phi(Q) formed inside the attention kernel (phase 2 long enough to
+    # hide them) versus precomputed, with and without phase-1 G products (d = 128
+    # merges the critical blocks' G into phase 1, d = 64 does not)
+    ("inkernel_zphi_merged", 1, 2, 64 * 40 + 9, 128, "sla", 3, 30, True, True),
+    ("inkernel_zphi_d64", 1, 2, 64 * 40 + 9, 64, "sla", 3, 30, True, True),
+    ("inkernel_zphi_sla2_kn", 1, 2, 64 * 40, 128, "sla2", 4, 24, True, True),
+    ("precomputed_zphi_merged_kn", 1, 2, 64 * 30 + 3, 128, "sla", 5, 4, True, True),
 ]
 
 
