@@ -16,9 +16,8 @@
 // blocks then read the same K/V tile at every step, which is loaded once.
 //
 // Warp roles (192 threads):
-//   warps 0-3  softmax / epilogue: one thread per query row (rows of block A
-//              in TMEM lanes 0-15 of each 32-lane quarter, block B in lanes
-//              16-31: two M=64 accumulators interleaved in the same columns);
+//   warps 0-3  softmax / epilogue: one thread per row of the pair (block A's
+//              64 rows in TMEM lanes 0-63, block B's in lanes 64-127);
 //   warp 4     TMA producer: Q tiles, then per step the K and V tiles of both
 //              blocks (phase 1; bf16 at d = 128 also phi(K) into the K slot
 //              once S has read it), then the phi(K) / V tiles of the remaining
@@ -27,17 +26,21 @@
 //              one elected lane issues each MMA and commit.
 // K tiles and V tiles travel in separate rings: a K slot is released as soon
 // as the S products that read it complete, a V slot after its PV product.
-// Phase 1 per step t: S = Q K_j^T (M=64, N=64) into one of two TMEM S
-// buffers; the softmax reads S and writes P (bf16) into one of two shared
-// buffers; O += P V_j (M=64, N=d). S(t+1) is issued before PV(t), so the
-// softmax of one step overlaps the tensor-core work of the next. O is
-// rescaled in TMEM only when a row maximum grows by more than 2^8 (the
-// exponent headroom of bf16 P and fp32 O). G += phi(K_j)^T V_j (M=d, N=d) over
+// Phase 1 per step t, over the 128-row pair [Q_A; Q_B] (M = 128 throughout):
+// S = [Q_A; Q_B] [K_jA; K_jB]^T (N = 128; A's rows keep columns 0-63, B's
+// 64-127; dense mode, where both blocks share K_j: N = 64) into one TMEM S
+// buffer; the softmax reads its row's 64 scores and writes P into the
+// block-diagonal P tile [128 rows][128 keys] (the other key half of a row stays
+// zero); O += P [V_jA; V_jB] (K = 128 keys, N = d). S(t+1) is issued as soon as
+// the softmax has read S(t), before PV(t). O is rescaled in TMEM only when a
+// row maximum grows by more than 2^8 (the exponent headroom of bf16 P and fp32
+// O). G += phi(K_j)^T V_j (M=d, N=d) over
 // E_i: for the critical blocks right after PV(t) on the V tile already
 // resident (bf16, d = 128), for the others in phase 2. Epilogue: phi(Q_i)
 // (precomputed, loaded over Q_i) dotted with Z_i (precomputed) gives the
-// denominator; H_i = H_tot - G in bf16 -> shared memory, num = phi(Q_i) H_i on
-// the tensor core, SLA's Y = O^l W likewise.
+// denominator; H_i = H_tot - G in bf16 -> shared memory, num = [phi(Q_A);
+// phi(Q_B)] H_X for X = A, B (M = 128, the rows of block X kept), SLA's
+// Y = O^l W as one M = 128 product.
 //
 // Every wait is bounded (about 2 s); an expired wait sets the device status
 // word to kDevTimeout and makes every later wait of the CTA return at once,
@@ -55,29 +58,34 @@ struct TcMaps {
   CUtensorMap qc, kc, vc;  // INT8 Q, K and e4m3 V codes (quantised sparse branch)
 };
 
+// Pair tiles: the 64 rows of block A followed by the 64 rows of block B (or
+// key blocks j_A, j_B), in 64-column SW128 sub-tiles of 128 rows x 128 B.
 template <int D>
 struct TcCfg {
   static constexpr int kSub = D / 64;          // 64-column sub-tiles of a row
   static constexpr int kTile = 64 * D * 2;     // bytes of a 64 x D bf16 tile
-  static constexpr int kNK = D == 128 ? 3 : 2; // K-ring slots (K_A, K_B | phiK_A, phiK_B)
-  static constexpr int kNV = 2;                // V-ring slots (V_A, V_B)
-  static constexpr int kPair = 2 * kTile;      // bytes of one ring slot
-  static constexpr int oQA = 0, oQB = kTile;   // Q (later phi(Q)) of blocks A, B
-  static constexpr int oP = 2 * kTile;         // P buffers: [2 steps][A, B] x 8 KB
-  static constexpr int oK = oP + 4 * 8192;
+  static constexpr int kSubS = 128 * 128;      // bytes of one 128-row sub-tile
+  static constexpr int kHalf = 64 * 128;       // offset of the B rows inside a sub-tile
+  static constexpr int kNK = D == 128 ? 3 : 2; // K-ring slots (K pair | phi(K) pair)
+  static constexpr int kNV = 2;                // V-ring slots (V pair)
+  static constexpr int kPair = kSub * kSubS;   // bytes of one ring slot (= 2 kTile)
+  static constexpr int oQ = 0;                 // Q pair tile (later phi(Q))
+  static constexpr int oP = kPair;             // P: [128 rows][128 keys] bf16, two 64-key sub-tiles
+  static constexpr int oK = oP + 2 * kSubS;
   static constexpr int oV = oK + kNK * kPair;
   static constexpr int kBytes = oV + kNV * kPair;
   // epilogue tiles reuse the rings once every loop product has completed
   static constexpr int kMat = D * D * 2;       // D x D bf16
   static constexpr int oHA = oK, oHB = oK + kMat, oW = oK + 2 * kMat;
-  static constexpr int oOlA = oK + 3 * kMat, oOlB = oOlA + kTile;
-  static_assert(oOlB + kTile <= kBytes, "epilogue tiles must fit in the rings");
-  // TMEM columns (fp32)
-  static constexpr int cS = 0;                 // S buffers [0,64) and [64,128)
+  static constexpr int oOl = oK + 3 * kMat;    // O^l pair tile
+  static_assert(oOl + kPair <= kBytes, "epilogue tiles must fit in the rings");
+  // TMEM columns (fp32); row i of the pair in lane i
+  static constexpr int cS = 0;                 // S: [128 rows][128 keys] (dense: 64)
   static constexpr int cO = 128;               // O: D columns
-  static constexpr int cG = 128 + D;           // G_A (D=128: G_B at cG + 128)
-  static constexpr int cNum = 0;               // num, after the loop
-  static constexpr int cY = cG;                // Y = O^l W, after G is consumed
+  static constexpr int cG = 128 + D;           // G_A (D=128: G_B at cG + 128; D=64: M=64 halves)
+  static constexpr int cNumA = 0;              // num of block A (over S, after the loop)
+  static constexpr int cNumB = D == 128 ? cG : 64;        // num of block B (over G_A / S)
+  static constexpr int cY = D == 128 ? cG + 128 : cG;     // Y = O^l W (over G_B / G)
   static constexpr uint32_t kTmemCols = D == 128 ? 512 : 256;
 };
 
@@ -85,7 +93,7 @@ enum Bar {
   bQFull = 0,
   bKFull0, bKFull1, bKFull2, bKEmpty0, bKEmpty1, bKEmpty2, bKDone0, bKDone1, bKDone2,
   bVFull0, bVFull1, bVEmpty0, bVEmpty1,
-  bSFull0, bSFull1, bSFree0, bSFree1, bPFull0, bPFull1, bPvDone0, bPvDone1,
+  bSFull, bSFree, bPFull, bPvDone,
   bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, bQFree, bPhiQFull, kNumBars
 };
 
@@ -184,10 +192,10 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   };
 
   const uint32_t sb = smem_u32(smem);
-  const uint32_t sQA = sb + C::oQA, sQB = sb + C::oQB, sP = sb + C::oP;
+  const uint32_t sQ = sb + C::oQ, sP = sb + C::oP;
   const uint32_t sK = sb + C::oK, sV = sb + C::oV;
   const uint32_t sHA = sb + C::oHA, sHB = sb + C::oHB, sW = sb + C::oW;
-  const uint32_t sOlA = sb + C::oOlA, sOlB = sb + C::oOlB;
+  const uint32_t sOl = sb + C::oOl;
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
@@ -201,12 +209,10 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       mbar_init(bar(bVFull0 + s), 1);
       mbar_init(bar(bVEmpty0 + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(bSFull0 + s), 1);
-      mbar_init(bar(bSFree0 + s), 128);
-      mbar_init(bar(bPFull0 + s), 128);
-      mbar_init(bar(bPvDone0 + s), 1);
-    }
+    mbar_init(bar(bSFull), 1);
+    mbar_init(bar(bSFree), 128);
+    mbar_init(bar(bPFull), 128);
+    mbar_init(bar(bPvDone), 1);
     mbar_init(bar(bTailDone), 1);
     mbar_init(bar(bHiFull), 1);
     mbar_init(bar(bNumFull), 1);
@@ -238,13 +244,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       }
       if constexpr (QNT) {  // INT8 Q codes: one 64 x 128-byte box per block
         mbar_expect_tx(bar(bQFull), 2 * 8192);
-        tma_load_3d(sQA, &maps.qc, bar(bQFull), 0, iA * 64, bh);
-        tma_load_3d(sQB, &maps.qc, bar(bQFull), 0, iB * 64, bh);
+        tma_load_3d(sQ, &maps.qc, bar(bQFull), 0, iA * 64, bh);
+        tma_load_3d(sQ + C::kHalf, &maps.qc, bar(bQFull), 0, iB * 64, bh);
       } else {
         mbar_expect_tx(bar(bQFull), 2 * C::kTile);
         for (int s = 0; s < C::kSub; ++s) {
-          tma_load_3d(sQA + s * 8192, &maps.q, bar(bQFull), s * 64, iA * 64, bh);
-          tma_load_3d(sQB + s * 8192, &maps.q, bar(bQFull), s * 64, iB * 64, bh);
+          tma_load_3d(sQ + s * C::kSubS, &maps.q, bar(bQFull), s * 64, iA * 64, bh);
+          tma_load_3d(sQ + s * C::kSubS + C::kHalf, &maps.q, bar(bQFull), s * 64, iB * 64, bh);
         }
       }
     }
@@ -258,8 +264,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       if (lane == 0) {
         mbar_expect_tx(bar(bPhiQFull), 2 * C::kTile);
         for (int s = 0; s < C::kSub; ++s) {
-          tma_load_3d(sQA + s * 8192, &maps.phiq, bar(bPhiQFull), s * 64, iA * 64, bh);
-          tma_load_3d(sQB + s * 8192, &maps.phiq, bar(bPhiQFull), s * 64, iB * 64, bh);
+          tma_load_3d(sQ + s * C::kSubS, &maps.phiq, bar(bPhiQFull), s * 64, iA * 64, bh);
+          tma_load_3d(sQ + s * C::kSubS + C::kHalf, &maps.phiq, bar(bPhiQFull), s * 64, iB * 64, bh);
         }
       }
       __syncwarp();
@@ -291,13 +297,14 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
             if (QNT && TK < nA) {
               mbar_expect_tx(bar(bKFull0 + st), codeBytes);
               tma_load_3d(slot, &maps.kc, bar(bKFull0 + st), 0, jA * 64, bh);
-              tma_load_3d(slot + C::kTile, &maps.kc, bar(bKFull0 + st), 0, jB * 64, bh);
+              tma_load_3d(slot + C::kHalf, &maps.kc, bar(bKFull0 + st), 0, jB * 64, bh);
             } else {
               const CUtensorMap* km = TK < nA ? &maps.k : &maps.phik;
               mbar_expect_tx(bar(bKFull0 + st), tileBytes);
               for (int s = 0; s < C::kSub; ++s) {
-                tma_load_3d(slot + s * 8192, km, bar(bKFull0 + st), s * 64, jA * 64, bh);
-                if (!dense) tma_load_3d(slot + C::kTile + s * 8192, km, bar(bKFull0 + st), s * 64, jB * 64, bh);
+                tma_load_3d(slot + s * C::kSubS, km, bar(bKFull0 + st), s * 64, jA * 64, bh);
+                if (!dense)
+                  tma_load_3d(slot + s * C::kSubS + C::kHalf, km, bar(bKFull0 + st), s * 64, jB * 64, bh);
               }
             }
           }
@@ -313,12 +320,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
             if (QNT && TV < nA) {
               mbar_expect_tx(bar(bVFull0 + st), codeBytes);
               tma_load_3d(slot, &maps.vc, bar(bVFull0 + st), 0, jA * 64, bh);
-              tma_load_3d(slot + C::kTile, &maps.vc, bar(bVFull0 + st), 0, jB * 64, bh);
+              tma_load_3d(slot + C::kHalf, &maps.vc, bar(bVFull0 + st), 0, jB * 64, bh);
             } else {
               mbar_expect_tx(bar(bVFull0 + st), tileBytes);
               for (int s = 0; s < C::kSub; ++s) {
-                tma_load_3d(slot + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jA * 64, bh);
-                if (!dense) tma_load_3d(slot + C::kTile + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jB * 64, bh);
+                tma_load_3d(slot + s * C::kSubS, &maps.v, bar(bVFull0 + st), s * 64, jA * 64, bh);
+                if (!dense)
+                  tma_load_3d(slot + s * C::kSubS + C::kHalf, &maps.v, bar(bVFull0 + st), s * 64, jB * 64, bh);
               }
             }
           }
@@ -333,8 +341,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       auto load_pair = [&](uint32_t slot, const CUtensorMap* m, uint32_t fb, int jA, int jB) {
         mbar_expect_tx(fb, 2 * C::kTile);
         for (int s = 0; s < C::kSub; ++s) {
-          tma_load_3d(slot + s * 8192, m, fb, s * 64, jA * 64, bh);
-          tma_load_3d(slot + C::kTile + s * 8192, m, fb, s * 64, jB * 64, bh);
+          tma_load_3d(slot + s * C::kSubS, m, fb, s * 64, jA * 64, bh);
+          tma_load_3d(slot + s * C::kSubS + C::kHalf, m, fb, s * 64, jB * 64, bh);
         }
       };
       uint32_t pe = (1u << C::kNK) - 1;  // KEmpty parity per slot (a slot's first fill passes)
@@ -406,54 +414,55 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     // The whole warp walks the loop (warp-uniform descriptors); the MMA and
     // commit helpers issue from one elected lane.
     {
-      constexpr uint32_t idS = idesc_bf16(64, 64, 0, 0);
-      constexpr uint32_t idPV = idesc_bf16(64, D, 0, 1);
+      // S, PV, num and Y run at M = 128 over the row pair (A rows, then B rows)
+      constexpr uint32_t idS = idesc_bf16(128, dense ? 64 : 128, 0, 0);
+      constexpr uint32_t idPV = idesc_bf16(128, D, 0, 1);
       constexpr uint32_t idG = idesc_bf16(D, D, 1, 1);
-      constexpr uint32_t idN = idesc_bf16(64, D, 0, 1);
-      constexpr uint32_t laneB = 16u << 16;  // block B's M=64 accumulators start at lane 16
-      const uint32_t tileB = dense ? 0u : uint32_t(C::kTile);  // dense: B reads A's tile
+      constexpr uint32_t idN = idesc_bf16(128, D, 0, 1);
+      constexpr uint32_t laneB = 16u << 16;  // D=64: G_B's M=64 accumulator starts at lane 16
       wait_w(bQFull, 0);
       tc_fence_after();
       auto issue_pv = [&](int tp) {
-        const int stv = tp % C::kNV, pb = tp & 1;
+        const int stv = tp % C::kNV;
         wait_w(bVFull0 + stv, (tp / C::kNV) & 1);
-        wait_w(bPFull0 + pb, (tp >> 1) & 1);
+        wait_w(bPFull, tp & 1);
         tc_fence_after();
         const uint32_t vslot = sV + stv * C::kPair;
-        const uint32_t pA = sP + pb * 16384, pB = pA + 8192;
         if constexpr (QNT) {
-          // A = P e4m3 [64 rows][64 keys], 64-byte swizzled rows; B = V codes
-          // [64 tokens][128 dims] MN-major; K = 32 keys per instruction
-          constexpr uint32_t idPV8 = idesc_e4m3(64, D, 0, 1);
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const uint32_t acc = (tp > 0 || k > 0) ? 1u : 0u;
-            mma_e4m3(tb + C::cO, sdesc(pA + k * 32, 16, 512, 4), sdesc(vslot + k * 4096, 8192, 1024), idPV8, acc);
-            mma_e4m3(tb + laneB + C::cO, sdesc(pB + k * 32, 16, 512, 4),
-                     sdesc(vslot + C::kTile + k * 4096, 8192, 1024), idPV8, acc);
-          }
-        } else {
+          // A = P e4m3 [128 rows][128 keys] (block diagonal: A rows over j_A's
+          // keys, B rows over j_B's), SW128; B = V codes [128 keys][128 dims]
+          // MN-major; K = 32 keys per instruction
+          constexpr uint32_t idPV8 = idesc_e4m3(128, D, 0, 1);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint32_t acc = (tp > 0 || k > 0) ? 1u : 0u;
-            mma_bf16(tb + C::cO, sdesc(pA + k * 32, 16, 1024), sdesc(vslot + k * 2048, 8192, 1024), idPV, acc);
-            mma_bf16(tb + laneB + C::cO, sdesc(pB + k * 32, 16, 1024),
-                     sdesc(vslot + tileB + k * 2048, 8192, 1024), idPV, acc);
+            mma_e4m3(tb + C::cO, sdesc(sP + k * 32, 16, 1024), sdesc(vslot + k * 4096, C::kSubS, 1024), idPV8, acc);
+          }
+        } else {
+          // A = P bf16 [128 rows][128 keys] block diagonal (dense: [128][64]),
+          // B = V pair [128 keys][D] MN-major
+          constexpr int nk = dense ? 4 : 8;
+#pragma unroll
+          for (int k = 0; k < nk; ++k) {
+            const uint32_t acc = (tp > 0 || k > 0) ? 1u : 0u;
+            mma_bf16(tb + C::cO, sdesc(sP + (k >> 2) * C::kSubS + (k & 3) * 32, 16, 1024),
+                     sdesc(vslot + k * 2048, C::kSubS, 1024), idPV, acc);
           }
         }
-        mma_commit(bar(bPvDone0 + pb));
+        mma_commit(bar(bPvDone));
         if (!merge) mma_commit(bar(bVEmpty0 + stv));  // merged: released after G
       };
       const uint32_t gA = tb + C::cG;
       const uint32_t gB = D == 128 ? tb + C::cG + 128 : tb + laneB + C::cG;
-      // G += phi(K_j)^T V_j for both blocks (M = N = D, MN-major operands)
+      // G += phi(K_j)^T V_j for both blocks (M = N = D, MN-major operands; the
+      // j_B rows sit kHalf into each sub-tile)
       auto issue_g = [&](uint32_t kslot, uint32_t vslot, bool first) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint32_t acc = (!first || k > 0) ? 1u : 0u;
-          mma_bf16(gA, sdesc(kslot + k * 2048, 8192, 1024), sdesc(vslot + k * 2048, 8192, 1024), idG, acc);
-          mma_bf16(gB, sdesc(kslot + C::kTile + k * 2048, 8192, 1024),
-                   sdesc(vslot + C::kTile + k * 2048, 8192, 1024), idG, acc);
+          mma_bf16(gA, sdesc(kslot + k * 2048, C::kSubS, 1024), sdesc(vslot + k * 2048, C::kSubS, 1024), idG, acc);
+          mma_bf16(gB, sdesc(kslot + C::kHalf + k * 2048, C::kSubS, 1024),
+                   sdesc(vslot + C::kHalf + k * 2048, C::kSubS, 1024), idG, acc);
         }
       };
       uint32_t kf = 0;  // KFull parity per slot
@@ -471,30 +480,27 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         mma_commit(bar(bVEmpty0 + stv));
       };
       for (int t = 0; t < nA; ++t) {
-        const int stk = t % C::kNK, b = t & 1;
+        const int stk = t % C::kNK;
         wait_kfull(stk);
-        wait_w(bSFree0 + b, ((t >> 1) & 1) ^ 1);
+        wait_w(bSFree, (t & 1) ^ 1);  // the softmax has read S(t-1)
         tc_fence_after();
         const uint32_t kslot = sK + stk * C::kPair;
         if constexpr (QNT) {
           // INT8 codes, one 128-byte swizzled row per token; K = 32 per instruction
-          constexpr uint32_t idS8 = idesc_s8(64, 64);
+          constexpr uint32_t idS8 = idesc_s8(128, 128);
 #pragma unroll
-          for (int k = 0; k < D / 32; ++k) {
-            mma_s8(tb + C::cS + b * 64, sdesc(sQA + k * 32, 16, 1024), sdesc(kslot + k * 32, 16, 1024), idS8, k > 0);
-            mma_s8(tb + laneB + C::cS + b * 64, sdesc(sQB + k * 32, 16, 1024),
-                   sdesc(kslot + C::kTile + k * 32, 16, 1024), idS8, k > 0);
-          }
+          for (int k = 0; k < D / 32; ++k)
+            mma_s8(tb + C::cS, sdesc(sQ + k * 32, 16, 1024), sdesc(kslot + k * 32, 16, 1024), idS8, k > 0);
         } else {
+          // [Q_A; Q_B] [K_jA; K_jB]^T (dense: [Q_A; Q_B] K_j^T); the A rows use
+          // columns 0-63, the B rows 64-127
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
-            mma_bf16(tb + C::cS + b * 64, sdesc(sQA + off, 16, 1024), sdesc(kslot + off, 16, 1024), idS, k > 0);
-            mma_bf16(tb + laneB + C::cS + b * 64, sdesc(sQB + off, 16, 1024),
-                     sdesc(kslot + tileB + off, 16, 1024), idS, k > 0);
+            const uint32_t off = (k >> 2) * C::kSubS + (k & 3) * 32;
+            mma_bf16(tb + C::cS, sdesc(sQ + off, 16, 1024), sdesc(kslot + off, 16, 1024), idS, k > 0);
           }
         }
-        mma_commit(bar(bSFull0 + b));
+        mma_commit(bar(bSFull));
         mma_commit(bar(merge ? bKDone0 + stk : bKEmpty0 + stk));  // merged: phi(K) refills the slot
         if (pre && t == nA - 1) mma_commit(bar(bQFree));          // Q tiles free for phi(Q)
         if (t > 0) {
@@ -519,12 +525,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       if (has_marg) {
         wait_w(bHiFull, 0);
         tc_fence_after();
+        // [phi(Q_A); phi(Q_B)] H_A and [phi(Q_A); phi(Q_B)] H_B: the A rows of
+        // the first and the B rows of the second are kept
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_bf16(tb + C::cNum, sdesc(sQA + off, 16, 1024), sdesc(sHA + k * 2048, D * 128, 1024), idN, k > 0);
-          mma_bf16(tb + laneB + C::cNum, sdesc(sQB + off, 16, 1024), sdesc(sHB + k * 2048, D * 128, 1024), idN,
-                   k > 0);
+          const uint32_t off = (k >> 2) * C::kSubS + (k & 3) * 32;
+          mma_bf16(tb + C::cNumA, sdesc(sQ + off, 16, 1024), sdesc(sHA + k * 2048, D * 128, 1024), idN, k > 0);
+          mma_bf16(tb + C::cNumB, sdesc(sQ + off, 16, 1024), sdesc(sHB + k * 2048, D * 128, 1024), idN, k > 0);
         }
         mma_commit(bar(bNumFull));
       }
@@ -534,10 +541,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
-          mma_bf16(tb + C::cY, sdesc(sOlA + off, 16, 1024), sdesc(sW + k * 2048, D * 128, 1024), idN, k > 0);
-          mma_bf16(tb + laneB + C::cY, sdesc(sOlB + off, 16, 1024), sdesc(sW + k * 2048, D * 128, 1024), idN,
-                   k > 0);
+          const uint32_t off = (k >> 2) * C::kSubS + (k & 3) * 32;
+          mma_bf16(tb + C::cY, sdesc(sOl + off, 16, 1024), sdesc(sW + k * 2048, D * 128, 1024), idN, k > 0);
         }
         mma_commit(bar(bYFull));
       }
@@ -548,14 +553,28 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     }
   } else {
     // --------------------------- softmax / epilogue ---------------------------
-    const int tid = threadIdx.x;  // 0..127
-    const bool isB = lane >= 16;
-    const int r = 16 * warp + (lane & 15);  // row inside the query block
+    const int tid = threadIdx.x;  // 0..127: row of the pair = TMEM lane
+    const bool isB = tid >= 64;   // warps 2-3
+    const int r = tid & 63;       // row inside the query block
     const int blk = isB ? iB : iA;
     const int grow = blk * 64 + r;          // row inside the head
     const bool store_row = grow < N && (!isB || validB);
     const uint32_t tq = tb + (uint32_t(32 * warp) << 16);  // this warp's TMEM lane quarter
-    unsigned char* Pbase = smem + C::oP + (isB ? 8192 : 0) + r * 128;
+    // this row's S columns and its P row (bf16: the 64-key sub-tile of its key
+    // block; e4m3: its half of a 128-byte row); the other half of the row stays zero
+    const int scol = dense ? 0 : (isB ? 64 : 0);
+    unsigned char* Prow = smem + C::oP + (QNT ? 0 : (dense || !isB ? 0 : C::kSubS)) + tid * 128;
+    if (!dense) {
+      if constexpr (QNT) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(Prow + (uint32_t((c + (isB ? 0 : 4)) ^ (tid & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+      } else {
+        unsigned char* other = smem + C::oP + (isB ? 0 : C::kSubS) + tid * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(other + (c << 4)) = make_uint4(0, 0, 0, 0);
+      }
+    }
     const float sl2 = a.scale_log2;
     // Only the block holding the last (partial) rows of the sequence has pad
     // keys; the lists are ascending, so it can only be the last step.
@@ -592,14 +611,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           named_bar(1, 128);
         }
       }
-      const int b = t & 1;
-      wait_w(bSFull0 + b, (t >> 1) & 1);
+      wait_w(bSFull, t & 1);
       tc_fence_after();
       float s[64];
       {
         float lo[32], hi[32];
-        tmem_ld32(tq + C::cS + b * 64, lo);
-        tmem_ld32(tq + C::cS + b * 64 + 32, hi);
+        tmem_ld32(tq + C::cS + scol, lo);
+        tmem_ld32(tq + C::cS + scol + 32, hi);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -608,7 +626,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(bSFree0 + b));
+      mbar_arrive(bar(bSFree));
       // scale of this step's scores into log2 units (quantised: int32 S times
       // s_q,i s_k,j)
       float cs = sl2;
@@ -637,7 +655,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       } else if (__any_sync(0xffffffffu, mx > m + kLazy)) {
         // some row of this warp grew by more than 2^kLazy: rescale the warp's O rows in TMEM
         // once PV(t-1) has landed in O
-        wait_w(bPvDone0 + ((t - 1) & 1), ((t - 1) >> 1) & 1);
+        wait_w(bPvDone, (t - 1) & 1);
         tc_fence_after();
         const float mnew = QNT ? ceilf(fmaxf(m, mx)) : fmaxf(m, mx);
         float corr;
@@ -672,29 +690,27 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         pk[i] = QNT ? pack_e4m3x2(p0 * pq_mul, p1 * pq_mul) : pack_bf16(p0, p1);
       }
       l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-      // P buffer b is free once PV(t-2) has completed
-      if (t >= 2) wait(bPvDone0 + b, ((t >> 1) & 1) ^ 1);
+      // the P buffer is free once PV(t-1) has completed
+      if (t >= 1) wait(bPvDone, (t - 1) & 1);
       if constexpr (QNT) {
-        // e4m3 P row: 64 bytes, 64-byte swizzle (16-byte chunk ^= (row / 2) % 4)
-        unsigned char* Prow = Pbase - r * 128 + b * 16384 + r * 64;
+        // e4m3 P: this row's 64 keys in its half of the 128-byte SW128 row
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(Prow + (uint32_t(c ^ ((r >> 1) & 3)) << 4)) =
+          *reinterpret_cast<uint4*>(Prow + (uint32_t((c + (isB ? 4 : 0)) ^ (tid & 7)) << 4)) =
               make_uint4(pk[8 * c] | (pk[8 * c + 1] << 16), pk[8 * c + 2] | (pk[8 * c + 3] << 16),
                          pk[8 * c + 4] | (pk[8 * c + 5] << 16), pk[8 * c + 6] | (pk[8 * c + 7] << 16));
       } else {
-        unsigned char* Prow = Pbase + b * 16384;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(Prow + (uint32_t(c ^ (r & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(Prow + (uint32_t(c ^ (tid & 7)) << 4)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(bPFull0 + b));
+      mbar_arrive(bar(bPFull));
     }
     // final O: the last PV (and every earlier product) has completed
-    wait_w(bPvDone0 + ((nA - 1) & 1), ((nA - 1) >> 1) & 1);
+    wait_w(bPvDone, (nA - 1) & 1);
     tc_fence_after();
     // quantised: undo the kPMul P scale and the V-scale fold
     const float inv_l = (QNT ? sv_max * (1.0f / kPMul) : 1.0f) / l;
@@ -712,11 +728,11 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       }
       named_bar(1, 128);  // zs complete
       wait_w(bPhiQFull, 0);
-      const unsigned char* Qrow = smem + (isB ? C::oQB : C::oQA);
+      const unsigned char* Qt = smem + C::oQ;
       den = 0.0f;
 #pragma unroll 4
       for (int c = 0; c < D / 8; ++c) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(Qrow + (c >> 3) * 8192 + sw128_chunk(r, c & 7));
+        const uint4 raw = *reinterpret_cast<const uint4*>(Qt + (c >> 3) * C::kSubS + sw128_chunk(tid, c & 7));
         const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -757,9 +773,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       // phi(Q) of this row, in place of the bf16 Q tile (K-major swizzled);
       // three passes over shared memory (max, sum, write) keep the row out of
       // registers
-      unsigned char* Qrow = smem + (isB ? C::oQB : C::oQA);
+      unsigned char* Qt = smem + C::oQ;
       auto qchunk = [&](int c) -> uint4* {
-        return reinterpret_cast<uint4*>(Qrow + (c >> 3) * 8192 + sw128_chunk(r, c & 7));
+        return reinterpret_cast<uint4*>(Qt + (c >> 3) * C::kSubS + sw128_chunk(tid, c & 7));
       };
       float qm = -INFINITY;
 #pragma unroll 4
@@ -800,7 +816,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       const float* ht = a.htot32 + size_t(bh) * D * D;
       // D=128: G rows c = TMEM lanes (M = 128), G_A and G_B in separate columns;
       // D=64:  G_A rows in lanes 0-15 of each quarter, G_B in lanes 16-31.
-      const int c = D == 128 ? tid : r;
+      const int c = D == 128 ? tid : 16 * warp + (lane & 15);
+      const bool g64B = lane >= 16;  // D=64: this lane holds G_B
       constexpr int kBlocksPerThread = D == 128 ? 2 : 1;
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -809,7 +826,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         for (int q = 0; q < 8; ++q) hv[q] = *reinterpret_cast<const float4*>(ht + size_t(c) * D + ch * 32 + 4 * q);
 #pragma unroll
         for (int X = 0; X < kBlocksPerThread; ++X) {
-          const bool xb = D == 128 ? X == 1 : isB;
+          const bool xb = D == 128 ? X == 1 : g64B;
           float g[32];
           tmem_ld32(tq + C::cG + (D == 128 ? X * 128 : 0) + ch * 32, g);
           tmem_wait_ld();
@@ -839,11 +856,11 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     __nv_bfloat16* orow = a.O + (size_t(bh) * (size_t(Nb) * 64) + grow) * D;
     if (use_y) {
       // O^l (bf16) -> K-major tile, then Y = O^l W on the tensor core
-      unsigned char* Olrow = smem + (isB ? C::oOlB : C::oOlA);
+      unsigned char* Olt = smem + C::oOl;
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
         float nm[32];
-        tmem_ld32(tq + C::cNum + ch * 32, nm);
+        tmem_ld32(tq + (isB ? C::cNumB : C::cNumA) + ch * 32, nm);
         tmem_wait_ld();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
@@ -852,7 +869,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
                                      pack_bf16(nm[q8 * 8 + 2] * inv_den, nm[q8 * 8 + 3] * inv_den),
                                      pack_bf16(nm[q8 * 8 + 4] * inv_den, nm[q8 * 8 + 5] * inv_den),
                                      pack_bf16(nm[q8 * 8 + 6] * inv_den, nm[q8 * 8 + 7] * inv_den));
-          *reinterpret_cast<uint4*>(Olrow + (e0 >> 6) * 8192 + sw128_chunk(r, (e0 & 63) >> 3)) = v;
+          *reinterpret_cast<uint4*>(Olt + (e0 >> 6) * C::kSubS + sw128_chunk(tid, (e0 & 63) >> 3)) = v;
         }
       }
       fence_async_smem();
@@ -867,7 +884,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       float o[32], x[32];
       tmem_ld32(tq + C::cO + ch * 32, o);
       if (use_y) tmem_ld32(tq + C::cY + ch * 32, x);
-      else if (has_marg) tmem_ld32(tq + C::cNum + ch * 32, x);
+      else if (has_marg) tmem_ld32(tq + (isB ? C::cNumB : C::cNumA) + ch * 32, x);
       tmem_wait_ld();
       float out[32];
 #pragma unroll
