@@ -89,6 +89,66 @@ def correction_flops(w):
     return w.B * w.H * w.Nb * (w.k_crit + w.k_neg) * 4.0 * 64 * 64 * w.d
 
 
+def executed_flops(w):
+    """Tensor FLOPs the attention kernel issues per launch. A CTA holds two
+    query blocks; per critical step S ([Q_A; Q_B][K_jA; K_jB]^T, N = 128) and
+    PV (block-diagonal P, K = 128 keys) run at M = 128, twice the algorithmic
+    products; G = phi(K_j)^T V_j per excluded block; phi(Q) H for both blocks'
+    H (twice the algorithmic product) and SLA's O^l W."""
+    BH, d = w.B * w.H, w.d
+    ctas = (w.Nb + 1) // 2
+    sparse = BH * ctas * w.k_crit * 2 * (2.0 * 128 * 128 * d)
+    linear = 0.0
+    if w.k_crit + w.k_neg < w.Nb:
+        linear = correction_flops(w) + BH * ctas * 2 * (2.0 * 128 * d * d)
+        if w.variant == "sla":
+            linear += BH * ctas * 2.0 * 128 * d * d
+    return sparse + linear
+
+
+def lowbit_peaks(bf16_burst):
+    """Dense INT8 and FP8 e4m3 GEMM throughput (TFLOP/s) of this GPU, 8192^3
+    through cuBLAS (torch._int_mm, torch._scaled_mm), 10 timed launches each;
+    None where the call is not available."""
+    import torch
+
+    n, reps = 8192, 10
+    out = {}
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        st.record()
+        for _ in range(reps):
+            fn()
+        en.record()
+        torch.cuda.synchronize()
+        return 2.0 * n ** 3 * reps / (st.elapsed_time(en) * 1e-3) / 1e12
+
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda")
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda").t()
+        out["i8_tops"] = round(timed(lambda: torch._int_mm(a, b)), 1)
+        del a, b
+    except Exception as e:  # noqa: BLE001
+        out["i8_tops"] = None
+        out["i8_error"] = str(e).splitlines()[0][:80]
+    try:
+        a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device="cuda")
+        out["fp8_tflops"] = round(timed(lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one,
+                                                                  out_dtype=torch.bfloat16)), 1)
+        del a, b
+    except Exception as e:  # noqa: BLE001
+        out["fp8_tflops"] = None
+        out["fp8_error"] = str(e).splitlines()[0][:80]
+    out["bf16_burst_ref"] = bf16_burst
+    return out
+
+
 def stage_bytes(w):
     """Bytes each memory-bound stage moves (reads + writes) in this design."""
     BH, N, Np, Nb, d = w.B * w.H, w.N, w.N_pad, w.Nb, w.d
@@ -361,8 +421,7 @@ def run_ours(args):
     roofline = {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": peak_tf,
                 "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
                 "traffic": ATTN_TRAFFIC.get(w.name), "kernel": "attention", "peak_kind": peak_kind,
-                "executed_tflops_incl_correction":
-                    round((attn_alg + correction_flops(w)) / (attn_ms * 1e-3) / 1e12, 2)}
+                "executed_tflops": round(executed_flops(w) / (attn_ms * 1e-3) / 1e12, 2)}
     in_bytes = 3 * w.B * w.H * w.N_pad * w.d * 2
     sb = stage_bytes(w)
     hbm = {k: {"ms": round(stages[k], 4), "GB/s": round(b / (stages[k] * 1e-3) / 1e9, 1),
@@ -413,16 +472,24 @@ def run_ours(args):
         msq /= args.steps
         f_lowbit, f_bf16 = attention_split_flops(wq)
         t_attn = stq["attention"] * 1e-3
-        # time the attention kernel's products need at the measured peaks: the
-        # INT8 / e4m3 sparse products at the 8-bit rate, the rest at bf16
-        t_min = (f_lowbit / LOWBIT_OVER_BF16 + f_bf16) / (peak_tf * 1e12)
+        # time the attention kernel's products need at the peaks: S on INT8 and
+        # PV on e4m3 (half the low-bit FLOPs each) at their measured cuBLAS rates
+        # scaled from burst to sustained like bf16, the rest at bf16 sustained
+        lb = lowbit_peaks(pk["bf16_tflops"])
+        to_sust = peak_tf / pk["bf16_tflops"]
+        p_i8 = (lb["i8_tops"] or LOWBIT_OVER_BF16 * pk["bf16_tflops"]) * to_sust
+        p_f8 = (lb["fp8_tflops"] or LOWBIT_OVER_BF16 * pk["bf16_tflops"]) * to_sust
+        t_min = (f_lowbit / 2 / (p_i8 * 1e12) + f_lowbit / 2 / (p_f8 * 1e12) + f_bf16 / (peak_tf * 1e12))
         res["quantized"] = {
             "workload": wq.name, "precision": wq.precision, "ms": round(msq, 4),
             "dense_eq_tflops": round(dense_eq_flops(wq) / (msq * 1e-3) / 1e12, 2),
             "attention_ms": round(stq["attention"], 4),
             "attention_tflops": round((f_lowbit + f_bf16) / t_attn / 1e12, 2),
             "attention_frac_of_mixed_peak": round(t_min / t_attn, 4),
-            "mixed_peak": f"8-bit products at {LOWBIT_OVER_BF16}x the {pk_kind} bf16 sustained peak",
+            "mixed_peak": {"i8_tops_sustained": round(p_i8, 1), "fp8_tflops_sustained": round(p_f8, 1),
+                           "bf16_tflops_sustained": peak_tf, "measured_burst": lb,
+                           "note": "cuBLAS 8192^3 burst x (bf16 sustained / bf16 burst); nominal 2x bf16 "
+                                   "where a measurement is missing"},
             "stages_ms": {k: round(v, 4) for k, v in stq.items()}}
         del devq
     if not args.no_e2e:
@@ -438,6 +505,55 @@ def run_ours(args):
         import torch.distributed as dist
 
         dist.destroy_process_group()
+
+
+SWEEP_N = (4096, 16384, 32768, 65536, 131072)
+SWEEP_SPARSITY = (90, 95, 97)
+
+
+def run_sweep(args):
+    """Sequence-length / sparsity sweep (B1 H12 d128): SLA (10 % negligible)
+    and SLA2 at 90/95/97 % sparsity, and the dense kernel, per N. One JSON line."""
+    import torch
+
+    import sparse_linear_attention_pool_b200 as sla
+
+    sla.load()
+    rows = []
+    for N in SWEEP_N:
+        base = W.sweep_workload(N, 95, "sla")
+        dev = device_inputs(W.make_inputs(base))  # Q, K, V depend on N and the seed only
+
+        def dev_for(w):
+            dv = dict(dev)
+            bf = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(  # noqa: E731
+                torch.bfloat16).cuda()
+            if w.variant == "sla2":
+                dv.update(w_proj=None, proj_q=bf(W.weight(w, "proj_q")), proj_k=bf(W.weight(w, "proj_k")),
+                          alpha=torch.from_numpy(W.alpha(w)).cuda())
+            else:
+                dv.update(w_proj=bf(W.weight(w, "w_proj")), proj_q=None, proj_k=None, alpha=None)
+            return dv
+
+        dense_steps = 3 if N >= 65536 else 5
+        dms = time_dense(sla, base, dev, dense_steps, 2)
+        rows.append({"N": N, "variant": "dense", "sparsity": 0, "ms": round(dms, 4),
+                     "dense_eq_tflops": round(dense_eq_flops(base) / (dms * 1e-3) / 1e12, 1)})
+        for variant in ("sla", "sla2"):
+            for sp in SWEEP_SPARSITY:
+                w = W.sweep_workload(N, sp, variant)
+                steps = max(5, min(args.steps, int(2e5 // max(N, 1))))
+                ms, st, _ = time_forward(sla, w, dev_for(w), steps, 3, 1, stage_timing=True)
+                ms /= steps
+                rows.append({"N": N, "variant": variant, "sparsity": sp, "k_crit": w.k_crit,
+                             "k_neg": w.k_neg, "ms": round(ms, 4),
+                             "attention_ms": round(st["attention"], 4),
+                             "dense_eq_tflops": round(dense_eq_flops(w) / (ms * 1e-3) / 1e12, 1),
+                             "speedup_vs_dense": round(dms / ms, 2)})
+                print(json.dumps(rows[-1]), file=sys.stderr, flush=True)
+        del dev
+    print(json.dumps({"sweep": rows, "shape": "B1 H12 d128", "data": "synthetic (seed 4)",
+                      "dtype": "bf16"}), flush=True)
 
 
 def run_reference(args):
@@ -484,11 +600,15 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-north-star", action="store_true")
     ap.add_argument("--no-quant", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="run the N / sparsity sweep instead of the benchmark line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
-    if args.impl == "reference":
+    if args.sweep:
+        run_sweep(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
