@@ -242,14 +242,22 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest x over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(w, world, ms_per_step):
+    """Whole-job dense-equivalent TFLOPS: every rank runs the workload once per
+    step (weak scaling), the step lasts the slowest rank's time."""
+    return dense_eq_flops(w) * world / (ms_per_step * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------------------
@@ -405,7 +413,7 @@ def run_ours(args):
     ms_total, stages, clk = time_forward(sla, w, dev, args.steps, args.warmup, world,
                                          stage_timing=True, clocks=clocks)
     ms = ms_total / args.steps
-    value = dense_eq_flops(w) * world / (ms * 1e-3) / 1e12
+    value = job_value(w, world, ms)
 
     # dominant kernel: the attention stage (tensor cores)
     attn_ms = stages["attention"]
