@@ -30,7 +30,8 @@ What the pages fix, and the readings taken where they are silent:
     ([SLA2-notes] section 2 and [SLA2-art]). Pooling is linear, so projecting
     the pooled vectors is the same map; the float32 specification pools first.
   * phi(x) = softmax over the head dimension ([SLA-walk] 3.2 "phi: Softmax";
-    [SLA2-notes] section 3 item 3).
+    [SLA2-notes] section 3 item 3); optionally elu(x) + 1 elementwise, the
+    alternative [SLA-sum] section 4 names and its Table 2 ablates.
   * Sparse branch: softmax attention restricted to the keys of critical
     blocks, scale 1/sqrt(d) ([SLA-sum] step 3; [SLA-walk] 2.2 online softmax).
   * Linear branch: H_i = sum_{Mc[i,j]=0} phi(K_j)^T V_j,
@@ -194,11 +195,25 @@ def mask_f64(q: np.ndarray, k: np.ndarray, N: int, k_crit: int, k_neg: int,
     return dict(scores=s, Mc=Mc, crit=crit, neg=neg)
 
 
-def phi(x: np.ndarray) -> np.ndarray:
-    """Feature map: softmax over the head dimension (last axis), max-subtracted."""
-    m = x.max(axis=-1, keepdims=True)
-    e = np.exp(x - m)
-    return e / e.sum(axis=-1, keepdims=True)
+PHI_KINDS = ("softmax", "elu1")
+
+
+def phi(x: np.ndarray, kind: str = "softmax") -> np.ndarray:
+    """Feature map of the linear branch.
+
+    'softmax': softmax over the head dimension (last axis), max-subtracted; the
+    map SLA and SLA2 use (SLA walkthrough, section 3.2).
+    'elu1': elu(x) + 1 elementwise, i.e. x + 1 for x > 0 and exp(x) otherwise;
+    the SLA structured summary (section 4) names it beside softmax and its
+    Table 2 ablates it as "SLA (elu+1)".
+    """
+    if kind == "softmax":
+        m = x.max(axis=-1, keepdims=True)
+        e = np.exp(x - m)
+        return e / e.sum(axis=-1, keepdims=True)
+    if kind == "elu1":
+        return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+    raise ValueError(f"unknown phi {kind!r}")
 
 
 def _block_tokens(blocks: np.ndarray, N: int) -> np.ndarray:
@@ -225,12 +240,12 @@ def sparse_branch(q: np.ndarray, k: np.ndarray, v: np.ndarray, Mc: np.ndarray, N
     return out
 
 
-def linear_terms(k: np.ndarray, v: np.ndarray, N: int):
+def linear_terms(k: np.ndarray, v: np.ndarray, N: int, phi_kind: str = "softmax"):
     """Per key block j: h_j = phi(K_j)^T V_j [d, d] and z_j = rowsum(phi(K_j)^T) [d],
     over the block's valid tokens."""
     Np, d = k.shape
     Nb = Np // BLOCK
-    pk = phi(k[:N])
+    pk = phi(k[:N], phi_kind)
     h = np.zeros((Nb, d, d), dtype=np.float64)
     z = np.zeros((Nb, d), dtype=np.float64)
     for j in range(Nb):
@@ -240,17 +255,18 @@ def linear_terms(k: np.ndarray, v: np.ndarray, N: int):
     return h, z
 
 
-def linear_branch(q: np.ndarray, k: np.ndarray, v: np.ndarray, Mc: np.ndarray, N: int) -> np.ndarray:
+def linear_branch(q: np.ndarray, k: np.ndarray, v: np.ndarray, Mc: np.ndarray, N: int,
+                  phi_kind: str = "softmax") -> np.ndarray:
     """O^l_i = phi(Q_i) H_i / (phi(Q_i) Z_i) with H_i, Z_i summed over the marginal
     blocks (Mc == 0) of row i. Rows whose marginal set is empty get O^l = 0. [N, d]."""
     Nb = Mc.shape[0]
     d = v.shape[1]
-    h, z = linear_terms(k, v, N)
+    h, z = linear_terms(k, v, N, phi_kind)
     marg = (Mc == 0).astype(np.float64)  # [Nb, Nb]; H_i = sum_j marg[i, j] h_j
     H = (marg @ h.reshape(Nb, d * d)).reshape(Nb, d, d)
     Z = marg @ z
     out = np.zeros((N, d), dtype=np.float64)
-    pq = phi(q[:N])
+    pq = phi(q[:N], phi_kind)
     for i in range(Nb):
         if not marg[i].any():
             continue
@@ -386,7 +402,8 @@ def forward_head(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, N: 
                  variant: str, k_crit: int, k_neg: int, softmax_scale: Optional[float] = None,
                  w_proj_bits: Optional[np.ndarray] = None, proj_q_bits: Optional[np.ndarray] = None,
                  proj_k_bits: Optional[np.ndarray] = None, alpha_h: Optional[float] = None,
-                 quantized: bool = False, with_f64_mask: bool = False) -> dict:
+                 quantized: bool = False, with_f64_mask: bool = False,
+                 phi_kind: str = "softmax") -> dict:
     """Forward pass of one (b, h) head from bf16 bit arrays [N_pad, d].
 
     Returns a dict with O [N, d] float64 (unrounded), O_s, O_l, the mask (Mc,
@@ -403,7 +420,7 @@ def forward_head(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, N: 
     Mc = m["Mc"]
     q, k, v = q32.astype(np.float64), k32.astype(np.float64), v32.astype(np.float64)
     o_s = sparse_branch(q, k, v, Mc, N, scale)
-    o_l = linear_branch(q, k, v, Mc, N)
+    o_l = linear_branch(q, k, v, Mc, N, phi_kind)
     if variant == "sla":
         W = bf16_to_f64(w_proj_bits) if w_proj_bits is not None else np.eye(d)
         comb = lambda a, b: combine_sla(a, b, W)  # noqa: E731
@@ -456,5 +473,5 @@ def forward(inputs, heads=None, quantized: bool = False) -> dict:
             k_crit=w.k_crit, k_neg=w.k_neg, w_proj_bits=inputs.w_proj,
             proj_q_bits=inputs.proj_q, proj_k_bits=inputs.proj_k,
             alpha_h=None if inputs.alpha is None else float(inputs.alpha[h]),
-            quantized=quantized)
+            quantized=quantized, phi_kind=w.phi)
     return res

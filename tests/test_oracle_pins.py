@@ -71,6 +71,28 @@ def test_phi_is_softmax_over_head_dim():
     assert np.isfinite(O.phi(x * 1e3)).all()
 
 
+def test_phi_elu1_is_elementwise_elu_plus_one():
+    # elu(x) + 1: x + 1 above zero, exp(x) at or below it; elementwise, so an
+    # entry depends on nothing else in its row, and rows are not normalised
+    x = RNG.standard_normal((6, 16)) * 3
+    p = O.phi(x, "elu1")
+    assert np.all(p > 0)
+    y = x.copy()
+    y[:, 5] += 7.0
+    q = O.phi(y, "elu1")
+    np.testing.assert_array_equal(np.delete(q, 5, axis=1), np.delete(p, 5, axis=1))
+    assert not np.allclose(p.sum(axis=-1), 1.0)
+    # continuity at 0 (value 1 from both sides), slope 1 above, exp ratios below
+    np.testing.assert_allclose(O.phi(np.array([-1e-12, 0.0, 1e-12]), "elu1"), 1.0, atol=1e-11)
+    pos = np.abs(x) + 0.25
+    np.testing.assert_allclose(O.phi(pos + 0.5, "elu1") - O.phi(pos, "elu1"), 0.5, atol=1e-13)
+    neg = -np.abs(x) - 0.25
+    np.testing.assert_allclose(O.phi(neg, "elu1") / O.phi(neg - 2.0, "elu1"), np.exp(2.0), rtol=1e-12)
+    assert O.phi(np.array([-800.0]), "elu1")[0] == 0.0 and O.phi(np.array([800.0]), "elu1")[0] == 801.0
+    with pytest.raises(ValueError):
+        O.phi(x, "relu")
+
+
 # ---------------------------------------------------------------------------
 # float32 specification of the mask scores
 # ---------------------------------------------------------------------------
@@ -227,8 +249,8 @@ def test_sparse_branch_masks_exactly_the_noncritical_blocks():
 # linear branch
 # ---------------------------------------------------------------------------
 
-def brute_force_linear(q, k, v, Mc, N):
-    pq, pk = O.phi(q[:N]), O.phi(k[:N])
+def brute_force_linear(q, k, v, Mc, N, phi_kind="softmax"):
+    pq, pk = O.phi(q[:N], phi_kind), O.phi(k[:N], phi_kind)
     out = np.zeros((N, v.shape[1]))
     for r in range(N):
         i = r // 64
@@ -243,12 +265,13 @@ def brute_force_linear(q, k, v, Mc, N):
     return out
 
 
-def test_linear_branch_matches_token_level_brute_force():
+@pytest.mark.parametrize("phi_kind", ["softmax", "elu1"])
+def test_linear_branch_matches_token_level_brute_force(phi_kind):
     N, d = 64 * 3 + 17, 12
     q, k, v = rand_head(N, d, scale=2), rand_head(N, d, scale=2), rand_head(N, d)
     Mc = np.array([[1, 0, -1, 0], [0, 0, 0, 0], [1, 1, 1, 0], [-1, 1, 1, 1]], dtype=np.int8)
-    got = O.linear_branch(q, k, v, Mc, N)
-    np.testing.assert_allclose(got, brute_force_linear(q, k, v, Mc, N), atol=1e-12)
+    got = O.linear_branch(q, k, v, Mc, N, phi_kind)
+    np.testing.assert_allclose(got, brute_force_linear(q, k, v, Mc, N, phi_kind), atol=1e-12)
     assert np.all(got[3 * 64:N] == 0.0)  # row 3 has no marginal block
 
 
@@ -268,6 +291,20 @@ def test_no_critical_block_gives_pure_linear_attention():
     A = pq @ pk.T
     r0 = O.forward_head(qb, kb, vb, N, variant="sla", k_crit=0, k_neg=0, w_proj_bits=eye)
     np.testing.assert_allclose(r0["O"], (A @ v) / A.sum(1, keepdims=True), atol=1e-12)
+
+
+def test_elu1_forward_without_critical_blocks_is_plain_linear_attention():
+    # the same identity with phi = elu + 1: every block marginal, W = I, so O is
+    # kernelised linear attention with k(q, k) = phi(q) . phi(k) over all tokens
+    N, d = 64 * 4 + 9, 8
+    qb, kb, vb = bits(rand_head(N, d, scale=2)), bits(rand_head(N, d, scale=2)), bits(rand_head(N, d))
+    r = O.forward_head(qb, kb, vb, N, variant="sla", k_crit=0, k_neg=0, w_proj_bits=bits(np.eye(d)),
+                       phi_kind="elu1")
+    q, k, v = (W.bf16_bits_to_f32(b)[:N].astype(np.float64) for b in (qb, kb, vb))
+    eq = np.where(q > 0, q + 1, np.exp(np.minimum(q, 0)))
+    ek = np.where(k > 0, k + 1, np.exp(np.minimum(k, 0)))
+    A = eq @ ek.T
+    np.testing.assert_allclose(r["O"], (A @ v) / A.sum(1, keepdims=True), atol=1e-12)
 
 
 def test_sla2_alpha_extremes_and_empty_marginal():
@@ -371,15 +408,16 @@ def test_quantized_branch_exact_when_inputs_sit_on_the_grids():
     # on its critical block are all equal to x (log2 units), so every P~ of the
     # row is c = 2^(x - ceil x) and every P code is e4m3(256 c): the branch is
     # the float64 sparse branch times e4m3(256 c) / (256 c), row by row.
+    rng = np.random.default_rng(2024)  # own stream: independent of test order
     d, N = 8, 128
-    q = RNG.integers(-20, 21, size=(N, d)).astype(np.float32)
+    q = rng.integers(-20, 21, size=(N, d)).astype(np.float32)
     q[0, 0] = 127
     q[64, 3] = -127
     k = np.zeros((N, d), dtype=np.float32)
     k[:64] = [127, 3, 0, 0, 0, 0, 0, 0]
     k[64:] = [-127, 5, 1, 0, 0, 0, 0, 0]
     grid = e4m3_grid()
-    v = (RNG.choice(grid[grid <= 448], size=(N, d)) * RNG.choice([-1, 1], size=(N, d))).astype(np.float32)
+    v = (rng.choice(grid[grid <= 448], size=(N, d)) * rng.choice([-1, 1], size=(N, d))).astype(np.float32)
     v[0, 0] = 448.0
     v[64, 1] = -448.0
     qb, kb, vb = bits(q), bits(k), bits(v)
@@ -392,7 +430,8 @@ def test_quantized_branch_exact_when_inputs_sit_on_the_grids():
     assert np.all((c > 0.5) & (c <= 1.0))
     factor = O.e4m3_round(256.0 * c) / (256.0 * c)
     assert np.any(factor != 1.0)  # the P step is really exercised
-    np.testing.assert_allclose(r["O_sq"], r["O_s"] * factor[:, None], rtol=1e-12, atol=1e-12)
+    # float64 rounding of the two sides only (one e4m3 step is 2^-4 relative)
+    np.testing.assert_allclose(r["O_sq"], r["O_s"] * factor[:, None], rtol=1e-10, atol=1e-12)
 
 
 def test_quantized_sparse_branch_error_is_quantisation_sized():

@@ -90,6 +90,7 @@ class Workload:
     cluster_scale: float
     seed: int
     pad_value: float = DEFAULT_PAD_VALUE
+    phi: str = "softmax"  # feature map of the linear branch: "softmax" | "elu1"
 
     @property
     def N_pad(self) -> int:
@@ -109,13 +110,13 @@ class Workload:
 
 
 def make_workload(name, B, H, N, d, variant, crit_pct=None, neg_pct=0.0, k_crit=None,
-                  k_neg=None, cluster_scale=2.0, seed=0, precision="bf16") -> Workload:
+                  k_neg=None, cluster_scale=2.0, seed=0, precision="bf16", phi="softmax") -> Workload:
     Nb = n_pad(N) // BLOCK
     if k_crit is None:
         k_crit, k_neg = block_counts(Nb, crit_pct, neg_pct)
     return Workload(name=name, B=B, H=H, N=N, d=d, variant=variant, precision=precision,
                     k_crit=int(k_crit), k_neg=int(k_neg or 0), cluster_scale=float(cluster_scale),
-                    seed=int(seed))
+                    seed=int(seed), phi=phi)
 
 
 # ---------------------------------------------------------------------------
