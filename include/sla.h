@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define SLA_ABI_VERSION 1
+#define SLA_ABI_VERSION 2 /* 2: sla_params.phi */
 #define SLA_BLOCK 64
 #define SLA_MAX_BLOCKS 4096 /* N <= 262144 */
 
@@ -81,6 +81,15 @@ typedef enum {
   SLA_PREC_I8QK_F8PV = 1  /* sparse branch with INT8 Q K^T and FP8 e4m3 P V */
 } sla_precision;
 
+/* Feature map phi of the linear branch, applied to every query and key row.
+ * SLA structured summary, section 4: phi is an activation such as softmax or
+ * ELU+1 (its Table 2 ablates both); the SLA walkthrough (section 3.2) and the
+ * SLA2 notes choose softmax. */
+typedef enum {
+  SLA_PHI_SOFTMAX = 0, /* softmax over the head dimension, max-subtracted */
+  SLA_PHI_ELU1 = 1     /* elu(x) + 1 elementwise: x + 1 for x > 0, exp(x) otherwise */
+} sla_phi;
+
 typedef struct sla_params {
   int B, H;            /* batch and heads (>= 1) */
   int N;               /* true sequence length (>= 1); tensors hold N_pad rows */
@@ -96,6 +105,7 @@ typedef struct sla_params {
   const void* proj_q;  /* SLA2 router: [d, d] bf16 device, qbar W_q; NULL = none (both or neither) */
   const void* proj_k;  /* SLA2 router: [d, d] bf16 device, kbar W_k */
   const float* alpha;  /* SLA2: [H] float32 device, per-head mixing weight; required for SLA2 */
+  int phi;             /* sla_phi; 0 (softmax) for the method as published */
 } sla_params;
 
 /* ABI version of the loaded library (SLA_ABI_VERSION at build time). */

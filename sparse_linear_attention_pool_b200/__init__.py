@@ -23,6 +23,7 @@ SLA_OK, SLA_ERR_INVALID_ARG, SLA_ERR_UNSUPPORTED, SLA_ERR_WORKSPACE, SLA_ERR_ALI
     SLA_ERR_CUDA, SLA_ERR_DEVICE_TIMEOUT, SLA_ERR_DEVICE_CHECK = range(8)
 VARIANTS = {"sla": 0, "sla2": 1}
 PRECISIONS = {"bf16": 0, "i8qk_f8pv": 1}
+PHIS = {"softmax": 0, "elu1": 1}  # feature map of the linear branch
 BLOCK = 64
 
 # every symbol include/sla.h declares
@@ -45,6 +46,7 @@ class Params(ctypes.Structure):
         ("softmax_scale", ctypes.c_float),
         ("w_proj", ctypes.c_void_p), ("proj_q", ctypes.c_void_p), ("proj_k", ctypes.c_void_p),
         ("alpha", ctypes.c_void_p),
+        ("phi", ctypes.c_int),
     ]
 
 
@@ -112,11 +114,13 @@ def _stream(stream) -> Optional[int]:
 
 
 def make_params(B, H, N, d, *, variant="sla", precision="bf16", k_crit, k_neg=0,
-                softmax_scale=0.0, w_proj=None, proj_q=None, proj_k=None, alpha=None) -> Params:
+                softmax_scale=0.0, w_proj=None, proj_q=None, proj_k=None, alpha=None,
+                phi="softmax") -> Params:
     return Params(B=B, H=H, N=N, d=d, block_q=BLOCK, block_kv=BLOCK,
                   variant=VARIANTS[variant], precision=PRECISIONS[precision],
                   k_crit=int(k_crit), k_neg=int(k_neg), softmax_scale=float(softmax_scale),
-                  w_proj=_ptr(w_proj), proj_q=_ptr(proj_q), proj_k=_ptr(proj_k), alpha=_ptr(alpha))
+                  w_proj=_ptr(w_proj), proj_q=_ptr(proj_q), proj_k=_ptr(proj_k), alpha=_ptr(alpha),
+                  phi=PHIS[phi])
 
 
 def validate(p: Params) -> int:
@@ -139,8 +143,8 @@ def allocate_workspace(p: Params, device=None):
 
 def forward(q, k, v, *, N: Optional[int] = None, variant: str = "sla", precision: str = "bf16",
             k_crit: Optional[int] = None, k_neg: int = 0, softmax_scale: float = 0.0, w_proj=None,
-            proj_q=None, proj_k=None, alpha=None, out=None, workspace=None, stream=None,
-            params=None):
+            proj_q=None, proj_k=None, alpha=None, phi: str = "softmax", out=None, workspace=None,
+            stream=None, params=None):
     """O = SLA / SLA2 forward of q, k, v ([B, H, N_pad, d] bf16 CUDA tensors).
 
     Returns (O, workspace); the workspace holds the mask and lists afterwards."""
@@ -152,7 +156,7 @@ def forward(q, k, v, *, N: Optional[int] = None, variant: str = "sla", precision
         raise ValueError("forward() needs k_crit or params")
     p = params or make_params(B, H, N, d, variant=variant, precision=precision, k_crit=k_crit,
                               k_neg=k_neg, softmax_scale=softmax_scale, w_proj=w_proj,
-                              proj_q=proj_q, proj_k=proj_k, alpha=alpha)
+                              proj_q=proj_q, proj_k=proj_k, alpha=alpha, phi=phi)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:

@@ -777,23 +777,29 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       auto qchunk = [&](int c) -> uint4* {
         return reinterpret_cast<uint4*>(Qt + (c >> 3) * C::kSubS + sw128_chunk(tid, c & 7));
       };
-      float qm = -INFINITY;
+      // phi = softmax over the row (max and sum passes first) or elu + 1
+      // elementwise (qm = 0 and qinv = 1 are unused then)
+      const bool elu1 = a.phi_elu1 != 0;
+      float qm = -INFINITY, qinv = 1.0f;
+      if (!elu1) {
 #pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 raw = *qchunk(c);
-        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 raw = *qchunk(c);
+          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) qm = fmaxf(qm, fmaxf(bf16_lo(wv[e]), bf16_hi(wv[e])));
-      }
-      float qs = 0.0f;
+          for (int e = 0; e < 4; ++e) qm = fmaxf(qm, fmaxf(bf16_lo(wv[e]), bf16_hi(wv[e])));
+        }
+        float qs = 0.0f;
 #pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 raw = *qchunk(c);
-        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 raw = *qchunk(c);
+          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) qs += expf(bf16_lo(wv[e]) - qm) + expf(bf16_hi(wv[e]) - qm);
+          for (int e = 0; e < 4; ++e) qs += expf(bf16_lo(wv[e]) - qm) + expf(bf16_hi(wv[e]) - qm);
+        }
+        qinv = 1.0f / qs;
       }
-      const float qinv = 1.0f / qs;
+      auto phi1 = [&](float x) { return elu1 ? (x > 0.0f ? x + 1.0f : expf(x)) : expf(x - qm) * qinv; };
       named_bar(1, 128);  // zs complete
       den = 0.0f;
 #pragma unroll 4
@@ -803,7 +809,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          pk[e] = pack_bf16(expf(bf16_lo(wv[e]) - qm) * qinv, expf(bf16_hi(wv[e]) - qm) * qinv);
+          pk[e] = pack_bf16(phi1(bf16_lo(wv[e])), phi1(bf16_hi(wv[e])));
           den += bf16_lo(pk[e]) * zs[isB][8 * c + 2 * e] + bf16_hi(pk[e]) * zs[isB][8 * c + 2 * e + 1];
         }
         *qchunk(c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);

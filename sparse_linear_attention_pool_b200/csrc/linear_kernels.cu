@@ -1,5 +1,6 @@
 // Linear-attention precompute (step 3 of the forward): phi(K) with
-// phi = softmax over the head dimension, the per-block column sums
+// phi = softmax over the head dimension (or, selected by the caller, elu + 1
+// elementwise: SLA structured summary, section 4), the per-block column sums
 // z_j = rowsum(phi(K_j)^T), and the per-head totals
 // H_tot = sum_j phi(K_j)^T V_j, Z_tot = sum_j z_j.
 //
@@ -30,8 +31,8 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
                                                       float* __restrict__ zblk,
                                                       float* __restrict__ hpart, float* __restrict__ zpart,
                                                       uint8_t* __restrict__ vcode,
-                                                      float* __restrict__ vscale, int N, int Npad,
-                                                      int Nb, int nchunk) {
+                                                      float* __restrict__ vscale, int phi_elu1, int N,
+                                                      int Npad, int Nb, int nchunk) {
   __shared__ float vred[8];
   constexpr int CPR = D / 8;    // 16-byte chunks per row
   constexpr int WPM = 128 / D;  // warps per 16-row m tile (1 for D=128, 2 for D=64)
@@ -98,22 +99,27 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
           x[0] = bf16_lo(raw);
           x[1] = bf16_hi(raw);
         }
-        float m = x[0];
+        if (phi_elu1) {  // elu(x) + 1, elementwise
 #pragma unroll
-        for (int e = 1; e < PL; ++e) m = fmaxf(m, x[e]);
+          for (int e = 0; e < PL; ++e) x[e] = x[e] > 0.0f ? x[e] + 1.0f : expf(x[e]);
+        } else {  // softmax over the row (the warp's 32 lanes)
+          float m = x[0];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        float s = 0.0f;
+          for (int e = 1; e < PL; ++e) m = fmaxf(m, x[e]);
 #pragma unroll
-        for (int e = 0; e < PL; ++e) {
-          x[e] = expf(x[e] - m);
-          s += x[e];
+          for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+          float s = 0.0f;
+#pragma unroll
+          for (int e = 0; e < PL; ++e) {
+            x[e] = expf(x[e] - m);
+            s += x[e];
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+          const float inv = 1.0f / s;
+#pragma unroll
+          for (int e = 0; e < PL; ++e) x[e] *= inv;
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        const float inv = 1.0f / s;
-#pragma unroll
-        for (int e = 0; e < PL; ++e) x[e] *= inv;
       } else {
 #pragma unroll
         for (int e = 0; e < PL; ++e) x[e] = 0.0f;
@@ -221,21 +227,21 @@ __global__ void __launch_bounds__(256) phik_hz_kernel(const __nv_bfloat16* __res
 template <int D>
 static cudaError_t launch_hz_t(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                                __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
-                               uint8_t* vcode, float* vscale, cudaStream_t s) {
+                               uint8_t* vcode, float* vscale, int phi_elu1, cudaStream_t s) {
   const int bytes = 5 * 64 * D * 2;
   cudaError_t e =
       cudaFuncSetAttribute(phik_hz_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
   phik_hz_kernel<D><<<dim3(L.nchunk, L.BH), 256, bytes, s>>>(K, V, phik, zblk, hpart, zpart, vcode, vscale,
-                                                            L.N, L.Npad, L.Nb, L.nchunk);
+                                                            phi_elu1, L.N, L.Npad, L.Nb, L.nchunk);
   return cudaGetLastError();
 }
 
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                            __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
-                           uint8_t* vcode, float* vscale, cudaStream_t s) {
-  return L.d == 128 ? launch_hz_t<128>(L, K, V, phik, zblk, hpart, zpart, vcode, vscale, s)
-                    : launch_hz_t<64>(L, K, V, phik, zblk, hpart, zpart, vcode, vscale, s);
+                           uint8_t* vcode, float* vscale, int phi_elu1, cudaStream_t s) {
+  return L.d == 128 ? launch_hz_t<128>(L, K, V, phik, zblk, hpart, zpart, vcode, vscale, phi_elu1, s)
+                    : launch_hz_t<64>(L, K, V, phik, zblk, hpart, zpart, vcode, vscale, phi_elu1, s);
 }
 
 // Fixed-order sum of n strided values: 8 interleaved partial sums (element i

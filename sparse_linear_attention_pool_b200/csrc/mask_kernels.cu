@@ -36,8 +36,8 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
                                                    float* __restrict__ qbar, float* __restrict__ kbar,
                                                    int8_t* __restrict__ qcode, int8_t* __restrict__ kcode,
                                                    float* __restrict__ qscale, float* __restrict__ kscale,
-                                                   __nv_bfloat16* __restrict__ phiq, int N, int Npad,
-                                                   int Nb) {
+                                                   __nv_bfloat16* __restrict__ phiq, int phi_elu1, int N,
+                                                   int Npad, int Nb) {
   constexpr int TPB = D / 8;        // threads per block row
   constexpr int BPC = 128 / TPB;    // blocks per CTA
   __shared__ float pooled[BPC][D];
@@ -82,22 +82,28 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
           x[2 * e] = bf16_lo(w[e]);
           x[2 * e + 1] = bf16_hi(w[e]);
         }
-        float m = x[0];
+        float inv = 1.0f;
+        if (phi_elu1) {  // elu(x) + 1, elementwise
 #pragma unroll
-        for (int e = 1; e < 8; ++e) m = fmaxf(m, x[e]);
+          for (int e = 0; e < 8; ++e) x[e] = x[e] > 0.0f ? x[e] + 1.0f : expf(x[e]);
+        } else {  // softmax over the row (the group's TPB lanes)
+          float m = x[0];
 #pragma unroll
-        for (int off = TPB / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(gmask, m, off));
-        // exp(x - m) as 2^(x log2 e - m log2 e) on the MUFU ex2 unit
-        const float ml = m * kLog2e;
-        float sum = 0.0f;
+          for (int e = 1; e < 8; ++e) m = fmaxf(m, x[e]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x[e] = ex2_approx(fmaf(x[e], kLog2e, -ml));
-          sum += x[e];
+          for (int off = TPB / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(gmask, m, off));
+          // exp(x - m) as 2^(x log2 e - m log2 e) on the MUFU ex2 unit
+          const float ml = m * kLog2e;
+          float sum = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            x[e] = ex2_approx(fmaf(x[e], kLog2e, -ml));
+            sum += x[e];
+          }
+#pragma unroll
+          for (int off = TPB / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(gmask, sum, off);
+          inv = 1.0f / sum;
         }
-#pragma unroll
-        for (int off = TPB / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(gmask, sum, off);
-        const float inv = 1.0f / sum;
         *reinterpret_cast<uint4*>(phiq + (size_t(bh) * Npad + size_t(blk) * kBlock + t) * D + c0) =
             make_uint4(pack_bf16(x[0] * inv, x[1] * inv), pack_bf16(x[2] * inv, x[3] * inv),
                        pack_bf16(x[4] * inv, x[5] * inv), pack_bf16(x[6] * inv, x[7] * inv));
@@ -177,24 +183,24 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
 cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                         const __nv_bfloat16* proj_q, const __nv_bfloat16* proj_k, float* qbar,
                         float* kbar, int8_t* qcode, int8_t* kcode, float* qscale, float* kscale,
-                        __nv_bfloat16* phiq, cudaStream_t s) {
+                        __nv_bfloat16* phiq, int phi_elu1, cudaStream_t s) {
   const int bpc = 128 / (L.d / 8);
   dim3 grid((L.Nb + bpc - 1) / bpc, L.BH, 2);
   // phi(Q) is a separate instantiation: the branch alone slows the plain pass
   if (L.d == 128) {
     if (phiq)
       pool_kernel<128, true><<<grid, 128, 0, s>>>(Q, K, proj_q, proj_k, qbar, kbar, qcode, kcode, qscale,
-                                                  kscale, phiq, L.N, L.Npad, L.Nb);
+                                                  kscale, phiq, phi_elu1, L.N, L.Npad, L.Nb);
     else
       pool_kernel<128, false><<<grid, 128, 0, s>>>(Q, K, proj_q, proj_k, qbar, kbar, qcode, kcode, qscale,
-                                                   kscale, nullptr, L.N, L.Npad, L.Nb);
+                                                   kscale, nullptr, 0, L.N, L.Npad, L.Nb);
   } else {
     if (phiq)
       pool_kernel<64, true><<<grid, 128, 0, s>>>(Q, K, proj_q, proj_k, qbar, kbar, qcode, kcode, qscale,
-                                                 kscale, phiq, L.N, L.Npad, L.Nb);
+                                                 kscale, phiq, phi_elu1, L.N, L.Npad, L.Nb);
     else
       pool_kernel<64, false><<<grid, 128, 0, s>>>(Q, K, proj_q, proj_k, qbar, kbar, qcode, kcode, qscale,
-                                                  kscale, nullptr, L.N, L.Npad, L.Nb);
+                                                  kscale, nullptr, 0, L.N, L.Npad, L.Nb);
   }
   return cudaGetLastError();
 }

@@ -39,6 +39,7 @@ sla_status check_params(const sla_params* p) {
     if ((p->proj_q == nullptr) != (p->proj_k == nullptr)) return SLA_ERR_INVALID_ARG;
   }
   if (p->precision == SLA_PREC_I8QK_F8PV && p->d != 128) return SLA_ERR_UNSUPPORTED;
+  if (p->phi != SLA_PHI_SOFTMAX && p->phi != SLA_PHI_ELU1) return SLA_ERR_INVALID_ARG;
   return SLA_OK;
 }
 
@@ -109,6 +110,7 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   float* kscale = L.quant ? reinterpret_cast<float*>(ws + L.kscale) : nullptr;
   float* vscale = L.quant ? reinterpret_cast<float*>(ws + L.vscale) : nullptr;
   const bool sla2 = p->variant == SLA_VARIANT_SLA2;
+  const int elu1 = p->phi == SLA_PHI_ELU1 ? 1 : 0;
 
   const int call = g_timer.used < g_timer.max_calls ? g_timer.used++ : -1;
   auto mark = [&](int k) {
@@ -118,13 +120,13 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   mark(0);
   if (e == cudaSuccess)
     e = launch_pool(L, bf(Q), bf(K), sla2 ? bf(p->proj_q) : nullptr, sla2 ? bf(p->proj_k) : nullptr,
-                    qbar, kbar, qcode, kcode, qscale, kscale, phiq, s);
+                    qbar, kbar, qcode, kcode, qscale, kscale, phiq, elu1, s);
   mark(1);
   if (e == cudaSuccess) e = launch_scores(L, qbar, kbar, scores, s);
   mark(2);
   if (e == cudaSuccess) e = launch_classify(L, scores, mc, crit, neg, s);
   mark(3);
-  if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, zpart, vcode, vscale, s);
+  if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, zpart, vcode, vscale, elu1, s);
   mark(4);
   if (e == cudaSuccess) e = launch_hz_reduce(L, zpart, hpart, htot32, ztot, s);
   if (e == cudaSuccess && L.pre)
@@ -144,6 +146,7 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
     a.zi = zi;
     a.ztot = ztot;
     a.zblk = zblk;
+    a.phi_elu1 = elu1;
     a.w_proj = sla2 ? nullptr : bf(p->w_proj);
     a.alpha = sla2 ? p->alpha : nullptr;
     a.status = reinterpret_cast<int*>(ws + L.status);

@@ -90,14 +90,14 @@ inline Layout make_layout(const sla_params& p) {
 cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bfloat16* K,
                         const __nv_bfloat16* proj_q, const __nv_bfloat16* proj_k, float* qbar,
                         float* kbar, int8_t* qcode, int8_t* kcode, float* qscale, float* kscale,
-                        __nv_bfloat16* phiq, cudaStream_t s);
+                        __nv_bfloat16* phiq, int phi_elu1, cudaStream_t s);
 cudaError_t launch_scores(const Layout& L, const float* qbar, const float* kbar, float* scores,
                           cudaStream_t s);
 cudaError_t launch_classify(const Layout& L, const float* scores, int8_t* mc, int32_t* crit,
                             int32_t* neg, cudaStream_t s);
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                            __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
-                           uint8_t* vcode, float* vscale, cudaStream_t s);
+                           uint8_t* vcode, float* vscale, int phi_elu1, cudaStream_t s);
 cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* hpart, float* htot32,
                              float* ztot, cudaStream_t s);
 // Z_i = Z_tot - sum of z_j over the excluded blocks of query block i
@@ -117,6 +117,7 @@ struct AttnArgs {
   const float* zi;             // [BH, Nb, d] Z_i, or null: formed in the kernel
   const float* ztot;           // [BH, d] Z_tot (in-kernel Z_i)
   const float* zblk;           // [BH, Nb, d] z_j (in-kernel Z_i)
+  int phi_elu1;                // phi = elu + 1 elementwise (else softmax over d)
   const __nv_bfloat16* w_proj; // [d, d] or null
   const float* alpha;          // [H] or null
   int* status;                 // device status word (null: not reported)

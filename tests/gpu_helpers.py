@@ -46,7 +46,7 @@ def run_library(sla, inp, dev=None, use_w=True, use_router=True, out_fill=None, 
     dev = dev or device_inputs(inp)
     B, H = inp.q.shape[:2]
     p = sla.make_params(B, H, w.N, w.d, variant=w.variant, precision=w.precision, k_crit=w.k_crit,
-                        k_neg=w.k_neg, w_proj=dev["w_proj"] if use_w else None,
+                        k_neg=w.k_neg, phi=w.phi, w_proj=dev["w_proj"] if use_w else None,
                         proj_q=dev["proj_q"] if use_router else None,
                         proj_k=dev["proj_k"] if use_router else None, alpha=dev["alpha"])
     out = torch.empty_like(dev["q"])
@@ -77,7 +77,8 @@ def oracle_head(inp, idx, use_w=True, use_router=True, quantized=False):
         w_proj_bits=inp.w_proj if use_w else None,
         proj_q_bits=inp.proj_q if use_router else None,
         proj_k_bits=inp.proj_k if use_router else None,
-        alpha_h=None if inp.alpha is None else float(inp.alpha[h]), quantized=quantized)
+        alpha_h=None if inp.alpha is None else float(inp.alpha[h]), quantized=quantized,
+        phi_kind=w.phi)
 
 
 def oracle_mask_only(inp, idx, use_router=True):

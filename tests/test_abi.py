@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sla_abi_version() == 1
+    assert lib.sla_abi_version() == 2
     for s in range(8):
         assert sla.status_string(s)
     assert "unknown" in sla.status_string(99)
@@ -63,9 +63,18 @@ def params(**kw):
     (dict(softmax_scale=-1.0), sla.SLA_ERR_INVALID_ARG),
     (dict(softmax_scale=float("nan")), sla.SLA_ERR_INVALID_ARG),
     (dict(variant="sla2", k_neg=0), sla.SLA_ERR_INVALID_ARG),  # SLA2 needs alpha
+    (dict(phi="elu1"), sla.SLA_OK),
 ])
 def test_validate(lib, kw, code):
     assert sla.validate(params(**kw)) == code
+
+
+def test_validate_rejects_unknown_phi(lib):
+    p = params()
+    for bad in (2, -1, 99):
+        p.phi = bad
+        assert sla.validate(p) == sla.SLA_ERR_INVALID_ARG
+        assert lib.sla_workspace_size(ctypes.byref(p)) == 0
 
 
 def test_bad_enum_and_block_size(lib):

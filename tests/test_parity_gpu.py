@@ -72,6 +72,27 @@ def test_edge_shapes(cuda_lib, case):
     check_all(cuda_lib, W.make_inputs(w), use_w=use_w, use_router=use_router)
 
 
+ELU1 = [
+    # phi = elu + 1 (SLA structured summary, section 4 and Table 2): every site
+    # that forms phi -- phi(K) in the linear precompute, phi(Q) precomputed in
+    # the pooling pass or formed in the attention epilogue, d = 64 and 128
+    # name, B, H, N, d, variant, k_crit, k_neg
+    ("elu1_sla_inkernel_merged", 1, 2, 64 * 40 + 9, 128, "sla", 3, 30),
+    ("elu1_sla_precomputed", 1, 2, 64 * 12 + 13, 128, "sla", 3, 2),
+    ("elu1_sla2_precomputed", 1, 2, 64 * 20 + 5, 128, "sla2", 4, 0),
+    ("elu1_d64_inkernel", 1, 2, 64 * 40 + 9, 64, "sla", 3, 30),
+    ("elu1_d64_sla2", 1, 1, 64 * 9 + 33, 64, "sla2", 2, 0),
+]
+
+
+@pytest.mark.parametrize("case", ELU1, ids=[c[0] for c in ELU1])
+def test_phi_elu1(cuda_lib, case):
+    name, B, H, N, d, variant, kc, kn = case
+    w = W.make_workload(name, B, H, N, d, variant, k_crit=kc, k_neg=kn, cluster_scale=2.0, seed=13,
+                        phi="elu1")
+    check_all(cuda_lib, W.make_inputs(w))
+
+
 def test_pad_rows_ignored_and_output_pad_untouched(cuda_lib):
     w = W.make_workload("pad", 1, 2, 64 * 8 + 23, 128, "sla", k_crit=2, k_neg=2, seed=5)
     a = run_library(cuda_lib, W.make_inputs(w))

@@ -99,6 +99,17 @@ def test_quantized_small(cuda_lib, case, record_property):
     check_outputs(inp, res, idxs, record_property)
 
 
+def test_quantized_phi_elu1(cuda_lib, record_property):
+    # phi = elu + 1 with the low-bit sparse branch (the linear branch stays bf16)
+    w = W.make_workload("q_elu1", 1, 2, 64 * 12 + 13, 128, "sla2", k_crit=2, k_neg=0, seed=33,
+                        precision=PREC, phi="elu1")
+    inp = W.make_inputs(w)
+    res = run_library(cuda_lib, inp)
+    assert res["status"] == 0
+    check_codes(cuda_lib, inp, res, [0, 1])
+    check_outputs(inp, res, [0, 1], record_property)
+
+
 @pytest.mark.slow
 def test_quantized_full_size_wan14b(cuda_lib, record_property):
     """The 40-head, 75,600-token SLA2 workload at 97 % sparsity: codes and
