@@ -54,7 +54,7 @@ namespace sla {
 using namespace tc;
 
 struct TcMaps {
-  CUtensorMap q, k, v, phik, w, phiq;
+  CUtensorMap q, k, v, phik, w, phiq, o;
   CUtensorMap qc, kc, vc;  // INT8 Q, K and e4m3 V codes (quantised sparse branch)
 };
 
@@ -555,10 +555,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     // --------------------------- softmax / epilogue ---------------------------
     const int tid = threadIdx.x;  // 0..127: row of the pair = TMEM lane
     const bool isB = tid >= 64;   // warps 2-3
-    const int r = tid & 63;       // row inside the query block
     const int blk = isB ? iB : iA;
-    const int grow = blk * 64 + r;          // row inside the head
-    const bool store_row = grow < N && (!isB || validB);
     const uint32_t tq = tb + (uint32_t(32 * warp) << 16);  // this warp's TMEM lane quarter
     // this row's S columns and its P row (bf16: the 64-key sub-tile of its key
     // block; e4m3: its half of a 128-byte row); the other half of the row stays zero
@@ -817,37 +814,45 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     }
     if (has_marg) {
       // H_i = H_tot - G_i -> bf16, MN-major tile [D rows c][D cols e]
-      wait_w(bTailDone, 0);
-      tc_fence_after();
-      const float* ht = a.htot32 + size_t(bh) * D * D;
       // D=128: G rows c = TMEM lanes (M = 128), G_A and G_B in separate columns;
       // D=64:  G_A rows in lanes 0-15 of each quarter, G_B in lanes 16-31.
       const int c = D == 128 ? tid : 16 * warp + (lane & 15);
       const bool g64B = lane >= 16;  // D=64: this lane holds G_B
       constexpr int kBlocksPerThread = D == 128 ? 2 : 1;
+      const float* hrow = a.htot32 + size_t(bh) * D * D + size_t(c) * D;
+      // H_tot row loads run one 32-column chunk ahead; chunk 0's before the
+      // wait for the last G product
+      float4 hv[8], hn[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hv[q] = *reinterpret_cast<const float4*>(hrow + 4 * q);
+      wait_w(bTailDone, 0);
+      tc_fence_after();
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
-        float4 hv[8];
+        if (ch + 1 < D / 32) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) hv[q] = *reinterpret_cast<const float4*>(ht + size_t(c) * D + ch * 32 + 4 * q);
+          for (int q = 0; q < 8; ++q) hn[q] = *reinterpret_cast<const float4*>(hrow + (ch + 1) * 32 + 4 * q);
+        }
+        float g[kBlocksPerThread][32];
+#pragma unroll
+        for (int X = 0; X < kBlocksPerThread; ++X) tmem_ld32(tq + C::cG + (D == 128 ? X * 128 : 0) + ch * 32, g[X]);
+        tmem_wait_ld();
 #pragma unroll
         for (int X = 0; X < kBlocksPerThread; ++X) {
           const bool xb = D == 128 ? X == 1 : g64B;
-          float g[32];
-          tmem_ld32(tq + C::cG + (D == 128 ? X * 128 : 0) + ch * 32, g);
-          tmem_wait_ld();
           unsigned char* Hbase = smem + (xb ? C::oHB : C::oHA);
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             const int e0 = ch * 32 + q8 * 8;
             const float4 h0 = hv[2 * q8], h1 = hv[2 * q8 + 1];
-            const uint4 v = make_uint4(pack_bf16(h0.x - g[q8 * 8 + 0], h0.y - g[q8 * 8 + 1]),
-                                       pack_bf16(h0.z - g[q8 * 8 + 2], h0.w - g[q8 * 8 + 3]),
-                                       pack_bf16(h1.x - g[q8 * 8 + 4], h1.y - g[q8 * 8 + 5]),
-                                       pack_bf16(h1.z - g[q8 * 8 + 6], h1.w - g[q8 * 8 + 7]));
+            const float* gx = g[X] + q8 * 8;
+            const uint4 v = make_uint4(pack_bf16(h0.x - gx[0], h0.y - gx[1]), pack_bf16(h0.z - gx[2], h0.w - gx[3]),
+                                       pack_bf16(h1.x - gx[4], h1.y - gx[5]), pack_bf16(h1.z - gx[6], h1.w - gx[7]));
             *reinterpret_cast<uint4*>(Hbase + (e0 >> 6) * (D * 128) + sw128_chunk(c, (e0 & 63) >> 3)) = v;
           }
         }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) hv[q] = hn[q];
       }
       fence_async_smem();
       tc_fence_before();
@@ -859,7 +864,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 
     const float alpha = MODE == kModeSLA2 ? a.alpha[h] : 0.0f;
     const float inv_den = 1.0f / den;
-    __nv_bfloat16* orow = a.O + (size_t(bh) * (size_t(Nb) * 64) + grow) * D;
+    // O is staged as a bf16 pair tile in the P region (free after the last PV)
+    // and written by TMA; the tensor map's row extent N drops the pad rows
+    unsigned char* Ot = smem + C::oP;
     if (use_y) {
       // O^l (bf16) -> K-major tile, then Y = O^l W on the tensor core
       unsigned char* Olt = smem + C::oOl;
@@ -899,13 +906,24 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         const float ol = use_y ? x[i] : (has_marg ? x[i] * inv_den : 0.0f);
         out[i] = MODE == kModeSLA2 ? alpha * os + (1.0f - alpha) * ol : os + ol;
       }
-      if (store_row) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-          dst[q8] = make_uint4(pack_bf16(out[8 * q8], out[8 * q8 + 1]), pack_bf16(out[8 * q8 + 2], out[8 * q8 + 3]),
-                               pack_bf16(out[8 * q8 + 4], out[8 * q8 + 5]), pack_bf16(out[8 * q8 + 6], out[8 * q8 + 7]));
+      for (int q8 = 0; q8 < 4; ++q8) {
+        const int e0 = ch * 32 + q8 * 8;
+        *reinterpret_cast<uint4*>(Ot + (e0 >> 6) * C::kSubS + sw128_chunk(tid, (e0 & 63) >> 3)) =
+            make_uint4(pack_bf16(out[8 * q8], out[8 * q8 + 1]), pack_bf16(out[8 * q8 + 2], out[8 * q8 + 3]),
+                       pack_bf16(out[8 * q8 + 4], out[8 * q8 + 5]), pack_bf16(out[8 * q8 + 6], out[8 * q8 + 7]));
       }
+    }
+    fence_async_smem();
+    named_bar(1, 128);
+    if (tid == 0) {
+      const uint32_t so = smem_u32(Ot);
+#pragma unroll
+      for (int s = 0; s < C::kSub; ++s) {
+        tma_store_3d(&maps.o, so + s * C::kSubS, s * 64, iA * 64, bh);
+        if (validB) tma_store_3d(&maps.o, so + s * C::kSubS + C::kHalf, s * 64, iB * 64, bh);
+      }
+      tma_store_commit_wait_read();
     }
   }
   tc_fence_before();
@@ -998,6 +1016,7 @@ cudaError_t launch_attention(const AttnArgs& a, int BH, int d, int mode, cudaStr
             map_rows(&maps.v, a.V, d, a.N, Npad, BH);
   if (ok && a.phik) ok = map_rows(&maps.phik, a.phik, d, Npad, Npad, BH);
   if (ok && a.phiq) ok = map_rows(&maps.phiq, a.phiq, d, a.N, Npad, BH);
+  if (ok) ok = map_rows(&maps.o, a.O, d, a.N, Npad, BH);
   if (ok && a.w_proj) ok = map_square(&maps.w, a.w_proj, d);
   const bool quant = a.qcode != nullptr;
   // the quantised branch's Q tiles hold INT8 codes: its phi(Q) must come precomputed
