@@ -12,9 +12,11 @@ Sources (cited by page title and section):
               formulas 1-4.
   [SLA-walk]  "SLA paper walkthrough: 95 % sparsity, 20x fewer FLOPs"
               (intelliparadigm.com), sections 1.2, 2.2 and 3.2.
-  [SLA2-notes] "SLA2 -- L3 Cross-Paper Synthesis" (zhaifeiyue.github.io), section 2.
+  [SLA2-notes] "SLA2 -- L3 Cross-Paper Synthesis" (zhaifeiyue.github.io),
+              sections 2 and 3.
   [SLA2-art]  popular article on SLA2, arXiv 2602.12675 (mcffsbgs.com),
-              paragraphs on the mixing formula, the router and quantisation.
+              paragraphs on the mixing formula, the router, quantisation and
+              the two-stage training.
 
 What the pages fix, and the readings taken where they are silent:
   * pool(.) is a mean over each 64-token block ([SLA-sum] formula 1,
@@ -47,6 +49,12 @@ What the pages fix, and the readings taken where they are silent:
   * Quantised sparse branch ([SLA2-art] quantisation paragraphs: Q, K, P, V
     go to low-bit values with scaling before and restoring after): see
     quantize_* and sparse_branch_quantized below for the exact scheme.
+  * SoftTop-k, the differentiable stand-in for Top-k in the first training
+    stage of SLA2's router ([SLA2-art] two-stage training; [SLA2-notes]
+    section 3): sigmoid((Pc_ij - lambda_i) / tau) on the router's Pc, the
+    matrix the hard Top-k ranks, with lambda_i found by bisection so that
+    every row sums to k = k_crit. The pages give no value for the
+    temperature tau: it is an argument.
 
 The bit-exact mask rests on one float32 operation order, emulated here op by
 op in NumPy float32 (each elementwise NumPy float32 operation is a single IEEE
@@ -193,6 +201,82 @@ def mask_f64(q: np.ndarray, k: np.ndarray, N: int, k_crit: int, k_neg: int,
     s = qbar @ kbar.T
     Mc, crit, neg = classify(s, k_crit, k_neg)
     return dict(scores=s, Mc=Mc, crit=crit, neg=neg)
+
+
+# ---------------------------------------------------------------------------
+# SoftTop-k router (stage-1 training of SLA2's router)
+# ---------------------------------------------------------------------------
+
+def compressed_softmax(scores: np.ndarray, scale: float) -> np.ndarray:
+    """Pc = softmax over each row of scale * s ([SLA-sum] formula 1), float64."""
+    x = np.asarray(scores, dtype=np.float64) * scale
+    e = np.exp(x - x.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def soft_topk(P: np.ndarray, k: int, tau: float):
+    """SoftTop-k of each row of P: M_ij = sigmoid((P_ij - lambda_i) / tau), with
+    lambda_i the root of sum_j M_ij = k ([SLA2-art] two-stage training: a
+    sigmoid with a temperature in place of Top-k; [SLA2-notes] section 3: a
+    binary search for lambda_i per row meets the row-sum constraint).
+
+    The row sum f(lambda) = sum_j sigmoid((P_ij - lambda) / tau) falls strictly
+    from n to 0, so the root is unique. Every term is >= k/n once
+    lambda <= min_j P_ij - tau logit(k/n), and <= k/n once
+    lambda >= max_j P_ij - tau logit(k/n): those two points bracket it. Bisection
+    halves the bracket until its midpoint equals an end (no float64 lies
+    between). The residual f - k is summed as (#{x_j > 0} - k) plus the signed
+    tails t_j = sigmoid(-|x_j|) (-t_j for x_j > 0, +t_j otherwise): each term
+    is then small and exact to rounding, where sigmoid(x_j) itself would
+    round to 1 and leave f flat around the root. k = n has no finite root:
+    M = 1 and lambda = -inf.
+    Returns (M [R, n] float64, lambda [R] float64).
+    """
+    P = np.asarray(P, dtype=np.float64)
+    R, n = P.shape
+    assert 1 <= k <= n and tau > 0
+    if k == n:
+        return np.ones((R, n)), np.full(R, -np.inf)
+
+    def split(lam):
+        x = (P - lam[:, None]) / tau
+        e = np.exp(-np.abs(x))
+        return x > 0, e / (1.0 + e)   # sigmoid(x) = 1 - t for x > 0, t otherwise
+
+    off = tau * np.log(k / (n - k))
+    lo = P.min(axis=1) - off
+    hi = P.max(axis=1) - off
+    for _ in range(4000):
+        mid = 0.5 * (lo + hi)
+        live = (mid > lo) & (mid < hi)
+        if not live.any():
+            break
+        pos, t = split(mid)
+        resid = (pos.sum(axis=1) - k) + np.where(pos, -t, t).sum(axis=1)
+        above = live & (resid > 0)   # f(mid) > k: the root lies right of mid
+        below = live & ~(resid > 0)
+        lo = np.where(above, mid, lo)
+        hi = np.where(below, mid, hi)
+    lam = 0.5 * (lo + hi)
+    pos, t = split(lam)
+    return np.where(pos, 1.0 - t, t), lam
+
+
+def router_soft_topk_head(q_bits: np.ndarray, k_bits: np.ndarray, N: int, k: int, tau: float,
+                          proj_q_bits: Optional[np.ndarray] = None,
+                          proj_k_bits: Optional[np.ndarray] = None,
+                          scale: Optional[float] = None) -> dict:
+    """Router forward of one head with SoftTop-k in place of the hard Top-k:
+    the pooled (and, for SLA2, projected) scores in the float32 specification,
+    Pc = softmax(scale s) with scale 1/sqrt(d) by default, then soft_topk(Pc, k, tau).
+    Returns dict(scores, Pc, M, lam)."""
+    d = q_bits.shape[1]
+    pq = bf16_to_f32(proj_q_bits) if proj_q_bits is not None else None
+    pk = bf16_to_f32(proj_k_bits) if proj_k_bits is not None else None
+    spec = mask_f32_spec(bf16_to_f32(q_bits), bf16_to_f32(k_bits), N, 1, 0, pq, pk)
+    Pc = compressed_softmax(spec["scores"], 1.0 / np.sqrt(d) if scale is None else scale)
+    M, lam = soft_topk(Pc, k, tau)
+    return dict(scores=spec["scores"], Pc=Pc, M=M, lam=lam)
 
 
 PHI_KINDS = ("softmax", "elu1")

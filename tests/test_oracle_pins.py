@@ -443,3 +443,89 @@ def test_quantized_sparse_branch_error_is_quantisation_sized():
                        k_crit=w.k_crit, k_neg=w.k_neg, w_proj_bits=inp.w_proj, quantized=True)
     err = r["O_sq"] - r["O_s"]
     assert 0 < np.linalg.norm(err) / np.linalg.norm(r["O_s"]) < 0.1
+
+
+# ---------------------------------------------------------------------------
+# SoftTop-k router
+# ---------------------------------------------------------------------------
+
+def test_soft_topk_uniform_row_closed_form():
+    # every entry equal: each M_ij = k / n and lambda = c - tau log(k / (n - k))
+    for n, k, tau, c in [(16, 3, 0.05, 0.0625), (512, 25, 1e-3, 1.0 / 512), (7, 6, 2.0, -3.0)]:
+        M, lam = O.soft_topk(np.full((2, n), c), k, tau)
+        np.testing.assert_allclose(M, k / n, rtol=1e-12)
+        np.testing.assert_allclose(lam, c - tau * math.log(k / (n - k)), rtol=1e-12, atol=1e-15)
+
+
+def test_soft_topk_two_entries_root_is_the_midpoint():
+    # n = 2, k = 1: sigmoid(a) + sigmoid(-a) = 1 puts lambda halfway between the entries
+    P = np.array([[0.9, 0.1], [0.25, 0.75], [0.5, 0.5]])
+    for tau in (0.01, 0.3, 5.0):
+        M, lam = O.soft_topk(P, 1, tau)
+        np.testing.assert_allclose(lam, P.mean(axis=1), rtol=1e-13)
+        want = 1.0 / (1.0 + np.exp(-(P[:, 0] - P[:, 1]) / (2 * tau)))
+        np.testing.assert_allclose(M[:, 0], want, rtol=1e-12)
+        np.testing.assert_allclose(M.sum(axis=1), 1.0, rtol=1e-13)
+
+
+def test_soft_topk_root_matches_brentq():
+    from scipy.optimize import brentq
+    from scipy.special import expit
+
+    rng = np.random.default_rng(77)
+    for n, k, tau in [(64, 3, 0.02), (300, 40, 1e-3), (33, 32, 0.5)]:
+        P = rng.dirichlet(np.full(n, 0.3), size=4)
+        M, lam = O.soft_topk(P, k, tau)
+        for r in range(P.shape[0]):
+            root = brentq(lambda x: expit((P[r] - x) / tau).sum() - k, -10.0, 10.0, xtol=1e-15, rtol=1e-15)
+            assert lam[r] == pytest.approx(root, rel=1e-10, abs=1e-13)
+        np.testing.assert_allclose(M.sum(axis=1), k, rtol=1e-10)
+        assert np.all((M >= 0) & (M <= 1))
+
+
+def test_soft_topk_small_temperature_is_the_hard_topk():
+    # distinct entries, gaps far above tau: the soft mask is the Top-k indicator
+    rng = np.random.default_rng(5)
+    n, k = 40, 6
+    P = np.stack([rng.permutation(n) for _ in range(5)]).astype(np.float64) / n
+    M, _ = O.soft_topk(P, k, 1e-4)
+    Mc, _, _ = O.classify(P, k, 0)
+    np.testing.assert_allclose(M, (Mc == 1).astype(np.float64), atol=1e-9)
+
+
+def test_soft_topk_shift_and_scale():
+    rng = np.random.default_rng(9)
+    P = rng.random((3, 50))
+    M, lam = O.soft_topk(P, 7, 0.05)
+    M2, lam2 = O.soft_topk(P + 0.375, 7, 0.05)
+    np.testing.assert_allclose(M2, M, atol=1e-12)
+    np.testing.assert_allclose(lam2, lam + 0.375, rtol=1e-12)
+    M3, lam3 = O.soft_topk(4.0 * P, 7, 0.2)
+    np.testing.assert_allclose(M3, M, atol=1e-12)
+    np.testing.assert_allclose(lam3, 4.0 * lam, rtol=1e-12)
+
+
+def test_soft_topk_every_block_selected():
+    M, lam = O.soft_topk(np.random.default_rng(2).random((2, 9)), 9, 0.1)
+    assert np.all(M == 1.0) and np.all(np.isneginf(lam))
+
+
+def test_router_pc_is_scaled_softmax_of_pooled_scores():
+    # integer block means pool exactly; Pc = softmax(qbar kbar^T / sqrt(d)) per row
+    from scipy.special import softmax
+
+    rng = np.random.default_rng(21)
+    Nb, d = 6, 16
+    qm = rng.integers(-2, 3, size=(Nb, d)).astype(np.float32)
+    km = rng.integers(-2, 3, size=(Nb, d)).astype(np.float32)
+    q = np.repeat(qm, 64, axis=0)
+    k = np.repeat(km, 64, axis=0)
+    r = O.router_soft_topk_head(bits(q), bits(k), Nb * 64, 2, 0.05)
+    s = qm.astype(np.float64) @ km.T.astype(np.float64)
+    np.testing.assert_array_equal(r["scores"], s)
+    np.testing.assert_allclose(r["Pc"], softmax(s / 4.0, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(r["M"].sum(axis=1), 2.0, rtol=1e-10)
+    # the router projections act on the pooled vectors
+    Wq = np.eye(d, dtype=np.float32)[::-1].copy()  # reverse the features of qbar
+    r2 = O.router_soft_topk_head(bits(q), bits(k), Nb * 64, 2, 0.05, bits(Wq), bits(np.eye(d, dtype=np.float32)))
+    np.testing.assert_array_equal(r2["scores"], qm[:, ::-1].astype(np.float64) @ km.T.astype(np.float64))
