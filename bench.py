@@ -331,6 +331,29 @@ def time_dense(sla, w, dev, steps, warmup):
     return start.elapsed_time(end) / steps
 
 
+ROUTER_TAU = 1e-2
+
+
+def time_router(sla, w, dev, steps, warmup, tau=ROUTER_TAU):
+    """ms per SoftTop-k router call (pooling with the router projections, pooled
+    scores, Pc and the per-row lambda / soft mask), on the current stream."""
+    import torch
+
+    p = sla.make_params(w.B, w.H, w.N, w.d, variant=w.variant, k_crit=w.k_crit, k_neg=w.k_neg,
+                        proj_q=dev["proj_q"], proj_k=dev["proj_k"], alpha=dev["alpha"])
+    ws = sla.allocate_workspace(p)
+    for _ in range(warmup):
+        sla.router_soft_topk(dev["q"], dev["k"], tau=tau, params=p, workspace=ws)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        sla.router_soft_topk(dev["q"], dev["k"], tau=tau, params=p, workspace=ws)
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps
+
+
 def time_e2e(sla, w, inp, steps, warmup, world):
     """Same metric through the C ABI with host buffers: each step copies Q, K, V
     from pinned host memory, runs the forward and copies O back."""
@@ -471,6 +494,8 @@ def run_ours(args):
                  "attention_tflops": round(attention_flops(w97) / (st97["attention"] * 1e-3) / 1e12, 2)}
         if "dense_baseline" in res:
             entry["speedup_vs_dense"] = round(res["dense_baseline"]["ms"] / ms97, 3)
+        entry["router_soft_topk"] = {"ms": round(time_router(sla, w97, dev97, 20, 3), 4), "tau": ROUTER_TAU,
+                                     "launches": 3}
         res["north_star_97"] = entry
         del dev97
     if not args.no_quant and rank == 0 and args.workload != QUANT_WORKLOAD:
@@ -498,7 +523,9 @@ def run_ours(args):
                            "bf16_tflops_sustained": peak_tf, "measured_burst": lb,
                            "note": "cuBLAS 8192^3 burst x (bf16 sustained / bf16 burst); nominal 2x bf16 "
                                    "where a measurement is missing"},
-            "stages_ms": {k: round(v, 4) for k, v in stq.items()}}
+            "stages_ms": {k: round(v, 4) for k, v in stq.items()},
+            "router_soft_topk": {"ms": round(time_router(sla, wq, devq, 10, 3), 4), "tau": ROUTER_TAU,
+                                 "launches": 3}}
         del devq
     if not args.no_e2e:
         e_ms, h2d, d2h = time_e2e(sla, w, inp, max(3, args.steps // 4), 2, world)

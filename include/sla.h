@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define SLA_ABI_VERSION 2 /* 2: sla_params.phi */
+#define SLA_ABI_VERSION 3 /* 2: sla_params.phi; 3: sla_router_soft_topk */
 #define SLA_BLOCK 64
 #define SLA_MAX_BLOCKS 4096 /* N <= 262144 */
 
@@ -157,6 +157,34 @@ sla_status sla_get_pooled(const sla_params* p, const void* workspace, float* qba
  * Returns SLA_ERR_INVALID_ARG for a bf16-precision parameter set. */
 sla_status sla_get_quantized(const sla_params* p, const void* workspace, int8_t* qcode, int8_t* kcode,
                              uint8_t* vcode, float* qscale, float* kscale, float* vscale, void* stream);
+
+/* SoftTop-k router forward, the differentiable stand-in for the hard Top-k in
+ * the first training stage of SLA2's router. Sources: SLA2 article
+ * (mcffsbgs.com), two-stage training paragraphs (a sigmoid with a temperature
+ * replaces Top-k); "SLA2 -- L3 Cross-Paper Synthesis" (zhaifeiyue.github.io),
+ * section 3 (lambda_i per row by binary search on the row-sum constraint);
+ * SLA structured summary (aipaper.cc), section 4, formula 1 (Pc).
+ *
+ * Runs step 1 of sla_forward (pooling; SLA2 with proj_q / proj_k: the router
+ * projections) and the pooled scores s_ij, then per row i:
+ *   Pc_ij = softmax_j(scale s_ij), scale = p->softmax_scale or 1/sqrt(d);
+ *   M_ij  = sigmoid((Pc_ij - lambda_i) / tau), lambda_i the unique root of
+ *           sum_j M_ij = k_crit, found in float32 inside a shrinking bracket
+ *           (Newton steps, bisection where a step would leave the bracket).
+ * k_crit = Nb gives M = 1 and lambda = -inf. p->k_neg, w_proj, alpha and phi
+ * are not used (p must still validate as for sla_forward).
+ *   Q, K      [B, H, N_pad, d] bf16 device inputs (as sla_forward).
+ *   tau       temperature: finite, > 0, and 1/tau finite.
+ *   m_soft    [B, H, Nb, Nb] float32 device output (required).
+ *   lambda    [B, H, Nb] float32 device output, or NULL.
+ *   pc        [B, H, Nb, Nb] float32 device output, or NULL.
+ *   workspace at least sla_workspace_size(p) bytes, 256-byte aligned; it
+ *             holds the pooled vectors and scores afterwards (sla_get_pooled).
+ * Errors: SLA_ERR_INVALID_ARG for a bad tau or a null Q, K or m_soft;
+ * otherwise as sla_forward. */
+sla_status sla_router_soft_topk(const void* Q, const void* K, const sla_params* p, float tau,
+                                float* m_soft, float* lambda, float* pc, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /* Synchronises the stream, then reads the device status word written by the
  * last sla_forward() on this workspace: SLA_OK, SLA_ERR_DEVICE_TIMEOUT if a

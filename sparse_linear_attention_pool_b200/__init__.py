@@ -30,7 +30,7 @@ BLOCK = 64
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate", "sla_workspace_size",
            "sla_forward", "sla_get_mask", "sla_get_pooled", "sla_read_device_status",
            "sla_dense_forward", "sla_stage_timing", "sla_stage_times", "sla_forward_noalloc",
-           "sla_get_quantized")
+           "sla_get_quantized", "sla_router_soft_topk")
 NOALLOC_WORKSPACE_BYTES = 32 << 20
 NUM_STAGES = 6
 STAGES = ("pool", "scores", "classify", "phik_hz", "hz_reduce", "attention")
@@ -81,6 +81,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sla_dense_forward": (i, [vp, vp, vp, vp, i, i, i, i, ctypes.c_float, vp]),
         "sla_forward_noalloc": (i, [vp, vp, vp, vp, P, vp]),
         "sla_get_quantized": (i, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "sla_router_soft_topk": (i, [vp, vp, P, ctypes.c_float, vp, vp, vp, vp, sz, vp]),
         "sla_stage_timing": (i, [i]),
         "sla_stage_times": (i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
     }
@@ -256,3 +257,24 @@ def get_quantized(p: Params, workspace, stream=None):
     _check(load().sla_get_quantized(ctypes.byref(p), _ptr(workspace), _ptr(qc), _ptr(kc), _ptr(vc),
                                     _ptr(qs), _ptr(ks), _ptr(vs), _stream(stream)), "sla_get_quantized")
     return qc, kc, vc, qs, ks, vs
+
+
+def router_soft_topk(q, k, *, tau: float, params: Params, workspace=None, want_pc: bool = False,
+                     stream=None):
+    """SoftTop-k router forward (sla_router_soft_topk): the pooled, router-projected
+    scores, Pc = softmax(scale s) per row and M = sigmoid((Pc - lambda) / tau) with
+    each row of M summing to params.k_crit.
+    Returns (M [B,H,Nb,Nb] float32, lambda [B,H,Nb] float32, Pc or None, workspace)."""
+    import torch
+
+    Nb = (params.N + BLOCK - 1) // BLOCK
+    dev = q.device
+    m = torch.empty((params.B, params.H, Nb, Nb), dtype=torch.float32, device=dev)
+    lam = torch.empty((params.B, params.H, Nb), dtype=torch.float32, device=dev)
+    pc = torch.empty_like(m) if want_pc else None
+    if workspace is None:
+        workspace = allocate_workspace(params, dev)
+    st = load().sla_router_soft_topk(_ptr(q), _ptr(k), ctypes.byref(params), float(tau), _ptr(m), _ptr(lam),
+                                     _ptr(pc), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sla_router_soft_topk")
+    return m, lam, pc, workspace

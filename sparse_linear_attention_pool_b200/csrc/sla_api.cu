@@ -169,6 +169,36 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
   return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
 }
 
+sla_status sla_router_soft_topk(const void* Q, const void* K, const sla_params* p, float tau,
+                                float* m_soft, float* lambda, float* pc, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  sla_status st = check_params(p);
+  if (st != SLA_OK) return st;
+  if (!Q || !K || !m_soft) return SLA_ERR_INVALID_ARG;
+  if (!(tau > 0.0f) || isinf(tau) || isinf(1.4426950408889634f / tau)) return SLA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(m_soft, 4) || (lambda && !aligned(lambda, 4)) ||
+      (pc && !aligned(pc, 4)))
+    return SLA_ERR_ALIGNMENT;
+  if ((p->proj_q && !aligned(p->proj_q, 16)) || (p->proj_k && !aligned(p->proj_k, 16)))
+    return SLA_ERR_ALIGNMENT;
+  const Layout L = make_layout(*p);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < L.total)
+    return SLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  auto bf = [](const void* x) { return static_cast<const __nv_bfloat16*>(x); };
+  float* qbar = reinterpret_cast<float*>(ws + L.qbar);
+  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
+  float* scores = reinterpret_cast<float*>(ws + L.scores);
+  const bool sla2 = p->variant == SLA_VARIANT_SLA2;
+  cudaError_t e = launch_pool(L, bf(Q), bf(K), sla2 ? bf(p->proj_q) : nullptr, sla2 ? bf(p->proj_k) : nullptr,
+                              qbar, kbar, nullptr, nullptr, nullptr, nullptr, nullptr, 0, s);
+  if (e == cudaSuccess) e = launch_scores(L, qbar, kbar, scores, s);
+  const float scale = p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / sqrtf(float(p->d));
+  if (e == cudaSuccess) e = launch_soft_topk(L, scores, m_soft, lambda, pc, scale, tau, s);
+  return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
+}
+
 sla_status sla_stage_timing(int max_calls) {
   if (max_calls < 0) return SLA_ERR_INVALID_ARG;
   for (cudaEvent_t ev : g_timer.events) cudaEventDestroy(ev);

@@ -103,6 +103,9 @@ cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* h
 // Z_i = Z_tot - sum of z_j over the excluded blocks of query block i
 cudaError_t launch_zi(const Layout& L, const int32_t* crit, const int32_t* neg, const float* zblk,
                       const float* ztot, float* zi, int* status, cudaStream_t s);
+// SoftTop-k of Pc = softmax(scale s) per row: m, lambda (may be null), pc (may be null)
+cudaError_t launch_soft_topk(const Layout& L, const float* scores, float* m, float* lambda, float* pc,
+                             float scale, float tau, cudaStream_t s);
 
 struct AttnArgs {
   const __nv_bfloat16* Q;
