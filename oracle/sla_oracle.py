@@ -1,4 +1,4 @@
-"""Float64 CPU oracle for the SLA / SLA2 sparse-linear attention forward pass.
+"""Float64 CPU oracle for the SLA / SLA2 sparse-linear attention forward and backward passes.
 
 TEST INFRASTRUCTURE. Only tests/, __graft_entry__.smoke() and bench.py's CPU
 baseline / reference leg may import this module. The product path (the CUDA
@@ -11,7 +11,7 @@ Sources (cited by page title and section):
               section 4 "Methodology", "Mathematical formulas & key details",
               formulas 1-4.
   [SLA-walk]  "SLA paper walkthrough: 95 % sparsity, 20x fewer FLOPs"
-              (intelliparadigm.com), sections 1.2, 2.2 and 3.2.
+              (intelliparadigm.com), sections 1.2, 2.2, 2.3 and 3.2.
   [SLA2-notes] "SLA2 -- L3 Cross-Paper Synthesis" (zhaifeiyue.github.io),
               sections 2 and 3.
   [SLA2-art]  popular article on SLA2, arXiv 2602.12675 (mcffsbgs.com),
@@ -55,6 +55,10 @@ What the pages fix, and the readings taken where they are silent:
     matrix the hard Top-k ranks, with lambda_i found by bisection so that
     every row sums to k = k_crit. The pages give no value for the
     temperature tau: it is an argument.
+  * Backward pass ([SLA-walk] section 2.3): the gradients of <dO, O> with the
+    mask held fixed (it is a hard Top-k of pooled scores). The sparse branch
+    is softmax attention over the critical keys, differentiated as such; the
+    linear branch by the chain rule through num / den, H_i, Z_i and phi.
 
 The bit-exact mask rests on one float32 operation order, emulated here op by
 op in NumPy float32 (each elementwise NumPy float32 operation is a single IEEE
@@ -369,6 +373,149 @@ def combine_sla(o_s: np.ndarray, o_l: np.ndarray, w_proj: np.ndarray) -> np.ndar
 def combine_sla2(o_s: np.ndarray, o_l: np.ndarray, alpha_h: float) -> np.ndarray:
     """SLA2: O = alpha O^s + (1 - alpha) O^l."""
     return alpha_h * o_s + (1.0 - alpha_h) * o_l
+
+
+# ---------------------------------------------------------------------------
+# backward pass (gradients of the forward above, the mask held fixed)
+# ---------------------------------------------------------------------------
+#
+# [SLA-walk] section 2.3: the sparse path follows the FlashAttention backward on
+# the Mc = 1 blocks; the linear path obtains the gradients of phi(Q), phi(K)
+# and V by the chain rule, accumulated block by block. The mask is a hard
+# Top-k of the pooled scores and has no gradient. Each function below is the
+# chain rule of the matching forward function written out; rows past N get
+# zero gradient.
+
+def phi_vjp(x: np.ndarray, dy: np.ndarray, kind: str = "softmax") -> np.ndarray:
+    """dx for y = phi(x) and upstream dy (row-wise Jacobian of the feature map)."""
+    if kind == "softmax":
+        y = phi(x, kind)
+        return y * (dy - (dy * y).sum(axis=-1, keepdims=True))
+    if kind == "elu1":
+        return np.where(x > 0, dy, dy * np.exp(np.minimum(x, 0.0)))
+    raise ValueError(f"unknown phi {kind!r}")
+
+
+def sparse_branch_backward(q, k, v, Mc, N, scale, do_s):
+    """Gradients of O^s for upstream do_s [N, d]: (dq, dk, dv) [N, d] each, and
+    lse [N], the natural-log normaliser log sum exp(scale q.k) of each row over
+    its critical keys (-inf for a row without critical blocks)."""
+    Nb = Mc.shape[0]
+    d = v.shape[1]
+    dq, dk, dv = (np.zeros((N, d)) for _ in range(3))
+    lse = np.full(N, -np.inf)
+    for i in range(Nb):
+        r0, r1 = i * BLOCK, min(N, (i + 1) * BLOCK)
+        keys = _block_tokens(np.nonzero(Mc[i] == 1)[0], N)
+        if keys.size == 0:
+            continue
+        s = (q[r0:r1] @ k[keys].T) * scale
+        mx = s.max(axis=1, keepdims=True)
+        e = np.exp(s - mx)
+        l = e.sum(axis=1, keepdims=True)
+        p = e / l
+        lse[r0:r1] = (mx + np.log(l))[:, 0]
+        g = do_s[r0:r1]
+        dv[keys] += p.T @ g
+        dp = g @ v[keys].T
+        ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+        dq[r0:r1] += scale * (ds @ k[keys])
+        dk[keys] += scale * (ds.T @ q[r0:r1])
+    return dq, dk, dv, lse
+
+
+def linear_branch_backward(q, k, v, Mc, N, do_l, phi_kind="softmax"):
+    """Gradients of O^l for upstream do_l [N, d]. With num = phi(Q_i) H_i,
+    den = phi(Q_i) Z_i and O^l = num / den:
+      dnum = do_l / den,  dden = -rowsum(do_l * O^l) / den,
+      dphi(Q_i) = dnum H_i^T + dden Z_i^T,
+      dH_i = phi(Q_i)^T dnum,  dZ_i = phi(Q_i)^T dden,
+    and, with A_j = sum of dH_i and b_j = sum of dZ_i over the rows i that have
+    j marginal, dphi(K_j) = V_j A_j^T + 1 b_j^T and dV_j = phi(K_j) A_j.
+    Returns (dq, dk, dv) [N, d] and den [N] (0 where the row has no marginal block)."""
+    Nb = Mc.shape[0]
+    d = v.shape[1]
+    h, z = linear_terms(k, v, N, phi_kind)
+    marg = (Mc == 0).astype(np.float64)
+    H = (marg @ h.reshape(Nb, d * d)).reshape(Nb, d, d)
+    Z = marg @ z
+    pq = phi(q[:N], phi_kind)
+    pk = phi(k[:N], phi_kind)
+    dpq = np.zeros((N, d))
+    dH = np.zeros((Nb, d, d))
+    dZ = np.zeros((Nb, d))
+    den_all = np.zeros(N)
+    for i in range(Nb):
+        if not marg[i].any():
+            continue
+        r0, r1 = i * BLOCK, min(N, (i + 1) * BLOCK)
+        num = pq[r0:r1] @ H[i]
+        den = pq[r0:r1] @ Z[i]
+        o = num / den[:, None]
+        den_all[r0:r1] = den
+        g = do_l[r0:r1]
+        dnum = g / den[:, None]
+        dden = -(g * o).sum(axis=1) / den
+        dpq[r0:r1] = dnum @ H[i].T + dden[:, None] * Z[i][None, :]
+        dH[i] = pq[r0:r1].T @ dnum
+        dZ[i] = pq[r0:r1].T @ dden
+    A = (marg.T @ dH.reshape(Nb, d * d)).reshape(Nb, d, d)
+    b = marg.T @ dZ
+    dpk = np.zeros((N, d))
+    dv = np.zeros((N, d))
+    for j in range(Nb):
+        t0, t1 = j * BLOCK, min(N, (j + 1) * BLOCK)
+        dpk[t0:t1] = v[t0:t1] @ A[j].T + b[j][None, :]
+        dv[t0:t1] = pk[t0:t1] @ A[j]
+    dq = phi_vjp(q[:N], dpq, phi_kind)
+    dk = phi_vjp(k[:N], dpk, phi_kind)
+    return dq, dk, dv, den_all
+
+
+def backward_head(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, do: np.ndarray, N: int, *,
+                  variant: str, k_crit: int, k_neg: int, softmax_scale: Optional[float] = None,
+                  w_proj_bits: Optional[np.ndarray] = None, proj_q_bits: Optional[np.ndarray] = None,
+                  proj_k_bits: Optional[np.ndarray] = None, alpha_h: Optional[float] = None,
+                  phi_kind: str = "softmax") -> dict:
+    """Backward pass of one (b, h) head: gradients of <dO, O> for upstream do
+    [N, d] (float64), O the forward_head output, with the mask of the forward.
+    SLA (O = O^s + O^l W): dO^s = dO, dO^l = dO W^T, dW = O^l^T dO.
+    SLA2 (O = a O^s + (1 - a) O^l): dO^s = a dO, dO^l = (1 - a) dO,
+    da = sum(dO * (O^s - O^l)).
+    Returns dQ, dK, dV [N, d], dW [d, d] (SLA) or dalpha (SLA2), the forward's
+    O_s, O_l, the sparse row normaliser lse [N], the linear denominator den [N]
+    and the mask."""
+    fw = forward_head(q_bits, k_bits, v_bits, N, variant=variant, k_crit=k_crit, k_neg=k_neg,
+                      softmax_scale=softmax_scale, w_proj_bits=w_proj_bits, proj_q_bits=proj_q_bits,
+                      proj_k_bits=proj_k_bits, alpha_h=alpha_h, phi_kind=phi_kind)
+    d = q_bits.shape[1]
+    scale = (1.0 / math.sqrt(d)) if not softmax_scale else float(softmax_scale)
+    W = None
+    if variant == "sla":
+        W = bf16_to_f64(w_proj_bits) if w_proj_bits is not None else np.eye(d)
+    res = backward_f64(bf16_to_f64(q_bits), bf16_to_f64(k_bits), bf16_to_f64(v_bits), fw["Mc"], do, N,
+                       variant=variant, scale=scale, W=W, alpha_h=alpha_h, phi_kind=phi_kind)
+    res.update(O=fw["O"], Mc=fw["Mc"], crit=fw["crit"], neg=fw["neg"])
+    return res
+
+
+def backward_f64(q, k, v, Mc, do, N, *, variant, scale, W=None, alpha_h=None, phi_kind="softmax") -> dict:
+    """backward_head on float64 [N_pad, d] arrays with a given mask."""
+    do = np.asarray(do, dtype=np.float64)[:N]
+    o_s = sparse_branch(q, k, v, Mc, N, scale)
+    o_l = linear_branch(q, k, v, Mc, N, phi_kind)
+    res = dict(O_s=o_s, O_l=o_l)
+    if variant == "sla":
+        do_s, do_l = do, do @ W.T
+        res["dW"] = o_l.T @ do
+    else:
+        a = float(alpha_h)
+        do_s, do_l = a * do, (1.0 - a) * do
+        res["dalpha"] = float((do * (o_s - o_l)).sum())
+    dq_s, dk_s, dv_s, lse = sparse_branch_backward(q, k, v, Mc, N, scale, do_s)
+    dq_l, dk_l, dv_l, den = linear_branch_backward(q, k, v, Mc, N, do_l, phi_kind)
+    res.update(dQ=dq_s + dq_l, dK=dk_s + dk_l, dV=dv_s + dv_l, lse=lse, den=den)
+    return res
 
 
 # ---------------------------------------------------------------------------

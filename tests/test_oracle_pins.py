@@ -529,3 +529,114 @@ def test_router_pc_is_scaled_softmax_of_pooled_scores():
     Wq = np.eye(d, dtype=np.float32)[::-1].copy()  # reverse the features of qbar
     r2 = O.router_soft_topk_head(bits(q), bits(k), Nb * 64, 2, 0.05, bits(Wq), bits(np.eye(d, dtype=np.float32)))
     np.testing.assert_array_equal(r2["scores"], qm[:, ::-1].astype(np.float64) @ km.T.astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# backward pass
+# ---------------------------------------------------------------------------
+
+def _bwd_case(variant, phi_kind, N=64 * 4 + 9, d=8, kc=2, kn=1, seed=0):
+    rng = np.random.default_rng(seed)
+    Np = 64 * ((N + 63) // 64)
+    q, k, v = (rng.standard_normal((Np, d)) for _ in range(3))
+    Nb = Np // 64
+    Mc, _, _ = O.classify(rng.standard_normal((Nb, Nb)), kc, kn if variant == "sla" else 0)
+    W = rng.standard_normal((d, d)) / math.sqrt(d)
+    alpha = 0.7
+    do = rng.standard_normal((N, d))
+    return q, k, v, Mc, W, alpha, do
+
+
+def _forward_fixed_mask(q, k, v, Mc, N, variant, W, alpha, phi_kind):
+    scale = 1.0 / math.sqrt(q.shape[1])
+    o_s = O.sparse_branch(q, k, v, Mc, N, scale)
+    o_l = O.linear_branch(q, k, v, Mc, N, phi_kind)
+    return O.combine_sla(o_s, o_l, W) if variant == "sla" else O.combine_sla2(o_s, o_l, alpha)
+
+
+@pytest.mark.parametrize("variant", ["sla", "sla2"])
+@pytest.mark.parametrize("phi_kind", ["softmax", "elu1"])
+def test_backward_matches_central_differences(variant, phi_kind):
+    N = 64 * 4 + 9
+    q, k, v, Mc, W, alpha, do = _bwd_case(variant, phi_kind, N)
+    scale = 1.0 / math.sqrt(q.shape[1])
+    g = O.backward_f64(q, k, v, Mc, do, N, variant=variant, scale=scale, W=W, alpha_h=alpha, phi_kind=phi_kind)
+    loss = lambda q_, k_, v_, W_, a_: float((do * _forward_fixed_mask(q_, k_, v_, Mc, N, variant, W_, a_,  # noqa: E731
+                                                                       phi_kind)).sum())
+    rng = np.random.default_rng(11)
+    eps = 1e-5
+    for name, grad in (("q", g["dQ"]), ("k", g["dK"]), ("v", g["dV"])):
+        delta = np.zeros_like(q)
+        delta[:N] = rng.standard_normal((N, q.shape[1]))
+        args = dict(q=q, k=k, v=v)
+        plus = dict(args, **{name: args[name] + eps * delta})
+        minus = dict(args, **{name: args[name] - eps * delta})
+        fd = (loss(plus["q"], plus["k"], plus["v"], W, alpha) - loss(minus["q"], minus["k"], minus["v"], W, alpha)) / (2 * eps)
+        an = float((grad * delta[:N]).sum())
+        assert an == pytest.approx(fd, rel=1e-6, abs=1e-8), name
+    if variant == "sla":
+        dW = rng.standard_normal(W.shape)
+        fd = (loss(q, k, v, W + eps * dW, alpha) - loss(q, k, v, W - eps * dW, alpha)) / (2 * eps)
+        assert float((g["dW"] * dW).sum()) == pytest.approx(fd, rel=1e-7, abs=1e-9)
+    else:
+        fd = (loss(q, k, v, W, alpha + eps) - loss(q, k, v, W, alpha - eps)) / (2 * eps)
+        assert g["dalpha"] == pytest.approx(fd, rel=1e-7, abs=1e-9)
+
+
+@pytest.mark.parametrize("variant,phi_kind,kc,kn", [("sla", "softmax", 2, 1), ("sla2", "softmax", 3, 0),
+                                                    ("sla", "elu1", 1, 2), ("sla", "softmax", 5, 0)])
+def test_backward_matches_autograd_of_token_level_formulation(variant, phi_kind, kc, kn):
+    """Independent formulation: masked dense softmax over critical keys and the
+    token-level linear attention sum_t phi(q).phi(k_t) v_t / sum_t phi(q).phi(k_t)
+    over marginal keys, differentiated by torch.autograd in float64."""
+    import torch
+
+    N = 64 * 4 + 9
+    q, k, v, Mc, W, alpha, do = _bwd_case(variant, phi_kind, N, kc=kc, kn=kn, seed=5)
+    d = q.shape[1]
+    g = O.backward_f64(q, k, v, Mc, do, N, variant=variant, scale=1.0 / math.sqrt(d), W=W, alpha_h=alpha,
+                       phi_kind=phi_kind)
+    blk = np.arange(N) // 64
+    crit_tok = torch.from_numpy(Mc[blk][:, blk] == 1)
+    marg_tok = torch.from_numpy(Mc[blk][:, blk] == 0).double()
+    T = lambda a: torch.tensor(a[:N], dtype=torch.float64, requires_grad=True)  # noqa: E731
+    tq, tk, tv = T(q), T(k), T(v)
+    tW = torch.tensor(W, requires_grad=True)
+    ta = torch.tensor(alpha, dtype=torch.float64, requires_grad=True)
+    s = (tq @ tk.T) / math.sqrt(d)
+    p = torch.softmax(s.masked_fill(~crit_tok, float("-inf")), dim=1)
+    o_s = torch.nan_to_num(p) @ tv
+    f = (lambda x: torch.softmax(x, dim=1)) if phi_kind == "softmax" else (lambda x: torch.where(x > 0, x + 1, torch.exp(torch.clamp(x, max=0.0))))
+    a = (f(tq) @ f(tk).T) * marg_tok
+    den = a.sum(dim=1, keepdim=True)
+    has = den > 0
+    o_l = torch.where(has, (a @ tv) / torch.where(has, den, torch.ones_like(den)), torch.zeros_like(o_s))
+    o = o_s + o_l @ tW if variant == "sla" else ta * o_s + (1 - ta) * o_l
+    (o * torch.from_numpy(do)).sum().backward()
+    np.testing.assert_allclose(g["dQ"], tq.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(g["dK"], tk.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(g["dV"], tv.grad.numpy(), rtol=1e-9, atol=1e-11)
+    if variant == "sla":
+        np.testing.assert_allclose(g["dW"], tW.grad.numpy(), rtol=1e-10, atol=1e-12)
+    else:
+        assert g["dalpha"] == pytest.approx(float(ta.grad), rel=1e-10)
+
+
+def test_backward_all_critical_is_softmax_attention_gradient():
+    """Every block critical (no linear branch): the gradients are those of exact
+    softmax attention, here torch's scaled_dot_product_attention in float64."""
+    import torch
+
+    N, d = 64 * 3, 16
+    rng = np.random.default_rng(8)
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    Mc = np.ones((3, 3), dtype=np.int8)
+    do = rng.standard_normal((N, d))
+    g = O.backward_f64(q, k, v, Mc, do, N, variant="sla2", scale=1.0 / math.sqrt(d), alpha_h=1.0)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq[None], tk[None], tv[None])[0]
+    (o * torch.from_numpy(do)).sum().backward()
+    for name, got, want in (("q", g["dQ"], tq.grad), ("k", g["dK"], tk.grad), ("v", g["dV"], tv.grad)):
+        np.testing.assert_allclose(got, want.numpy(), rtol=1e-9, atol=1e-11, err_msg=name)
+    assert np.isfinite(g["lse"]).all()
+    np.testing.assert_allclose(g["lse"], np.log(np.exp(q @ k.T / math.sqrt(d)).sum(axis=1)), rtol=1e-12)
