@@ -84,6 +84,18 @@ def attention_split_flops(w):
     return sparse, attention_flops(w) - sparse
 
 
+def backward_flops(w):
+    """Algorithmic tensor FLOPs of one backward: per critical pair S, dP, dQ,
+    dK and dV (5 x 2 x 64 x 64 x d); for the linear branch dphi(Q) = dnum H^T,
+    dH = phi(Q)^T dnum, dV += phi(K) A, dphi(K) = V A^T and h_j = phi(K)^T V
+    (5 x 2 N d^2); SLA also dO W^T and dW (2 x 2 N d^2)."""
+    BH = w.B * w.H
+    sparse = BH * w.Nb * w.k_crit * 5 * 2.0 * 64 * 64 * w.d
+    linear = BH * 5 * 2.0 * w.N * w.d * w.d if w.k_crit + w.k_neg < w.Nb else 0.0
+    proj = BH * 2 * 2.0 * w.N * w.d * w.d if w.variant == "sla" else 0.0
+    return sparse + linear + proj
+
+
 def correction_flops(w):
     """Extra tensor FLOPs executed for H_i = H_tot - sum over excluded blocks."""
     return w.B * w.H * w.Nb * (w.k_crit + w.k_neg) * 4.0 * 64 * 64 * w.d
@@ -334,6 +346,46 @@ def time_dense(sla, w, dev, steps, warmup):
 ROUTER_TAU = 1e-2
 
 
+def time_backward(sla, w, dev, steps, warmup):
+    """(ms per sla_backward call, ms per sla_forward_train call, ms per dense
+    FlashAttention backward of the same shape through torch's
+    scaled_dot_product_attention, for context; None where unavailable)."""
+    import torch
+
+    p = sla.make_params(w.B, w.H, w.N, w.d, variant=w.variant, k_crit=w.k_crit, k_neg=w.k_neg, phi=w.phi,
+                        w_proj=dev["w_proj"], proj_q=dev["proj_q"], proj_k=dev["proj_k"], alpha=dev["alpha"])
+    do = torch.randn_like(dev["q"])
+    out, saved, fws = sla.forward_train(dev["q"], dev["k"], dev["v"], params=p)
+    bws = torch.empty(sla.backward_workspace_size(p), dtype=torch.uint8, device=dev["q"].device)
+
+    def timed(fn, n, wu):
+        for _ in range(wu):
+            fn()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record()
+        for _ in range(n):
+            fn()
+        end.record()
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / n
+
+    bwd = timed(lambda: sla.backward(dev["q"], dev["k"], dev["v"], do, params=p, saved=saved, fwd_workspace=fws,
+                                     workspace=bws), steps, warmup)
+    fwd = timed(lambda: sla.forward_train(dev["q"], dev["k"], dev["v"], params=p, out=out, workspace=fws,
+                                          saved=saved), steps, warmup)
+    dense = None
+    try:
+        qd, kd, vd = (dev[x][:, :, :w.N].detach().clone().requires_grad_(True) for x in ("q", "k", "v"))
+        with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.FLASH_ATTENTION):
+            od = torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
+            g = torch.randn_like(od)
+            dense = timed(lambda: torch.autograd.grad(od, (qd, kd, vd), g, retain_graph=True), 3, 1)
+    except Exception:  # no flash backend for this shape / build
+        dense = None
+    return bwd, fwd, dense
+
+
 def time_router(sla, w, dev, steps, warmup, tau=ROUTER_TAU):
     """ms per SoftTop-k router call (pooling with the router projections, pooled
     scores, Pc and the per-row lambda / soft mask), on the current stream."""
@@ -477,6 +529,14 @@ def run_ours(args):
            "gpu_launches": (7 if w.k_crit + w.k_neg < w.Nb else 6) * args.steps,
            "clocks": clk}
 
+    if not args.no_backward and rank == 0 and w.precision == "bf16":
+        bms, fms, dms = time_backward(sla, w, dev, 10, 2)
+        res["backward"] = {"ms": round(bms, 4), "forward_train_ms": round(fms, 4),
+                           "tflops": round(backward_flops(w) / (bms * 1e-3) / 1e12, 2),
+                           "dense_flash_backward_ms": None if dms is None else round(dms, 4),
+                           "speedup_vs_dense_backward": None if dms is None else round(dms / bms, 3),
+                           "note": "sla_backward (mask fixed) after one sla_forward_train; dense = torch "
+                                   "scaled_dot_product_attention flash backward, same shape, for context"}
     if not args.no_dense and rank == 0:
         dense_ms = time_dense(sla, w, dev, args.dense_steps, 2)
         res["dense_baseline"] = {"ms": round(dense_ms, 4),
@@ -496,6 +556,11 @@ def run_ours(args):
             entry["speedup_vs_dense"] = round(res["dense_baseline"]["ms"] / ms97, 3)
         entry["router_soft_topk"] = {"ms": round(time_router(sla, w97, dev97, 20, 3), 4), "tau": ROUTER_TAU,
                                      "launches": 3}
+        b97, f97, d97 = time_backward(sla, w97, dev97, 10, 2)
+        entry["backward"] = {"ms": round(b97, 4), "forward_train_ms": round(f97, 4),
+                             "tflops": round(backward_flops(w97) / (b97 * 1e-3) / 1e12, 2),
+                             "dense_flash_backward_ms": None if d97 is None else round(d97, 4),
+                             "speedup_vs_dense_backward": None if d97 is None else round(d97 / b97, 3)}
         res["north_star_97"] = entry
         del dev97
     if not args.no_quant and rank == 0 and args.workload != QUANT_WORKLOAD:
@@ -633,6 +698,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--dense-steps", type=int, default=5)
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-north-star", action="store_true")
     ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--sweep", action="store_true",

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define SLA_ABI_VERSION 3 /* 2: sla_params.phi; 3: sla_router_soft_topk */
+#define SLA_ABI_VERSION 4 /* 2: sla_params.phi; 3: sla_router_soft_topk; 4: training forward, backward */
 #define SLA_BLOCK 64
 #define SLA_MAX_BLOCKS 4096 /* N <= 262144 */
 
@@ -132,6 +132,48 @@ sla_status sla_validate(const sla_params* p);
  *   stream    cudaStream_t as void*. */
 sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, const sla_params* p,
                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Training: the backward pass.
+ * Source: SLA walkthrough (intelliparadigm.com), section 2.3: the sparse path
+ * takes the FlashAttention backward on the Mc = 1 blocks, the linear path the
+ * gradients of phi(Q), phi(K) and V by the chain rule, block by block.
+ *
+ * Activations a training forward keeps for sla_backward (device buffers owned
+ * by the caller; rows N .. N_pad-1 are not written). */
+typedef struct sla_saved {
+  void* o_s;   /* [B, H, N_pad, d] bf16: the sparse branch O^s */
+  void* o_l;   /* [B, H, N_pad, d] bf16: the linear branch O^l (SLA: before W) */
+  float* lse;  /* [B, H, N_pad] float32: log sum_t exp(scale q.k_t) over the row's critical keys */
+  float* den;  /* [B, H, N_pad] float32: phi(q) . Z_i, 0 where the row has no marginal block */
+} sla_saved;
+
+/* sla_forward (same arguments and result) that also writes the activations of
+ * `saved` (every pointer required, 16-byte aligned bf16 / 4-byte float32).
+ * bf16 precision only (SLA_ERR_UNSUPPORTED otherwise). Keep the workspace and
+ * `saved` unchanged until sla_backward has run on them. */
+sla_status sla_forward_train(const void* Q, const void* K, const void* V, void* O, const sla_params* p,
+                             const sla_saved* saved, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace sla_backward() needs (0 for invalid parameters). */
+size_t sla_backward_workspace_size(const sla_params* p);
+
+/* Gradients of <dO, O> for the forward of sla_forward_train with the block
+ * mask held fixed (a hard Top-k has no gradient; no gradient reaches the
+ * router projections or the pooling).
+ *   Q, K, V, dO   [B, H, N_pad, d] bf16 device inputs; rows >= N of dO are ignored.
+ *   p, saved      the parameters and activations of the training forward.
+ *   fwd_workspace its workspace (mask, block lists, phi(K), z_j, H_tot, Z_tot).
+ *   dQ, dK, dV    [B, H, N_pad, d] bf16 device outputs; rows >= N are written as 0.
+ *   dW            SLA: [d, d] float32 device output, sum over batch and heads of
+ *                 O^l^T dO (the gradient of W); may be NULL. Must be NULL for SLA2.
+ *   dalpha        SLA2: [H] float32 device output, sum over the batch of
+ *                 dO . (O^s - O^l); may be NULL. Must be NULL for SLA.
+ *   workspace     at least sla_backward_workspace_size(p) bytes, 256-byte aligned.
+ * bf16 precision only. The result is deterministic (no floating-point atomics). */
+sla_status sla_backward(const void* Q, const void* K, const void* V, const void* dO, const sla_params* p,
+                        const sla_saved* saved, const void* fwd_workspace, size_t fwd_workspace_bytes, void* dQ,
+                        void* dK, void* dV, float* dW, float* dalpha, void* workspace, size_t workspace_bytes,
+                        void* stream);
 
 /* Copies the compressed mask and block lists of the last sla_forward() that
  * used this workspace (stream-ordered, device to device; any output may be NULL).

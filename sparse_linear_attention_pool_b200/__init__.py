@@ -30,7 +30,8 @@ BLOCK = 64
 EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate", "sla_workspace_size",
            "sla_forward", "sla_get_mask", "sla_get_pooled", "sla_read_device_status",
            "sla_dense_forward", "sla_stage_timing", "sla_stage_times", "sla_forward_noalloc",
-           "sla_get_quantized", "sla_router_soft_topk")
+           "sla_get_quantized", "sla_router_soft_topk", "sla_forward_train", "sla_backward_workspace_size",
+           "sla_backward")
 NOALLOC_WORKSPACE_BYTES = 32 << 20
 NUM_STAGES = 6
 STAGES = ("pool", "scores", "classify", "phik_hz", "hz_reduce", "attention")
@@ -48,6 +49,12 @@ class Params(ctypes.Structure):
         ("alpha", ctypes.c_void_p),
         ("phi", ctypes.c_int),
     ]
+
+
+class Saved(ctypes.Structure):
+    """Mirror of struct sla_saved (device pointers)."""
+    _fields_ = [("o_s", ctypes.c_void_p), ("o_l", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("den", ctypes.c_void_p)]
 
 
 class SLAError(RuntimeError):
@@ -82,6 +89,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sla_forward_noalloc": (i, [vp, vp, vp, vp, P, vp]),
         "sla_get_quantized": (i, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "sla_router_soft_topk": (i, [vp, vp, P, ctypes.c_float, vp, vp, vp, vp, sz, vp]),
+        "sla_forward_train": (i, [vp, vp, vp, vp, P, ctypes.POINTER(Saved), vp, sz, vp]),
+        "sla_backward_workspace_size": (sz, [P]),
+        "sla_backward": (i, [vp, vp, vp, vp, P, ctypes.POINTER(Saved), vp, sz, vp, vp, vp, vp, vp, vp, sz, vp]),
         "sla_stage_timing": (i, [i]),
         "sla_stage_times": (i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
     }
@@ -278,3 +288,55 @@ def router_soft_topk(q, k, *, tau: float, params: Params, workspace=None, want_p
                                      _ptr(pc), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "sla_router_soft_topk")
     return m, lam, pc, workspace
+
+
+def forward_train(q, k, v, *, params: Params, out=None, workspace=None, saved=None, stream=None):
+    """sla_forward_train: the forward pass that also keeps what the backward reads.
+    Returns (O, saved dict of tensors o_s, o_l, lse, den, workspace)."""
+    import torch
+
+    B, H, Np, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = allocate_workspace(params, q.device)
+    if saved is None:
+        saved = dict(o_s=torch.empty_like(q), o_l=torch.empty_like(q),
+                     lse=torch.empty((B, H, Np), dtype=torch.float32, device=q.device),
+                     den=torch.empty((B, H, Np), dtype=torch.float32, device=q.device))
+    sv = Saved(o_s=_ptr(saved["o_s"]), o_l=_ptr(saved["o_l"]), lse=_ptr(saved["lse"]), den=_ptr(saved["den"]))
+    st = load().sla_forward_train(_ptr(q), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(params), ctypes.byref(sv),
+                                  _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sla_forward_train")
+    return out, saved, workspace
+
+
+def backward_workspace_size(p: Params) -> int:
+    n = load().sla_backward_workspace_size(ctypes.byref(p))
+    if n == 0:
+        _check(validate(p), "sla_backward_workspace_size")
+    return n
+
+
+def backward(q, k, v, do, *, params: Params, saved: dict, fwd_workspace, want_param_grad: bool = True,
+             workspace=None, stream=None):
+    """sla_backward: gradients of <dO, O> for the forward of forward_train (mask fixed).
+    Returns (dQ, dK, dV, dW or dalpha or None, workspace)."""
+    import torch
+
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    sla2 = params.variant == VARIANTS["sla2"]
+    dW = dalpha = None
+    if want_param_grad:
+        if sla2:
+            dalpha = torch.empty(params.H, dtype=torch.float32, device=q.device)
+        else:
+            dW = torch.empty((params.d, params.d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(backward_workspace_size(params), dtype=torch.uint8, device=q.device)
+    sv = Saved(o_s=_ptr(saved["o_s"]), o_l=_ptr(saved["o_l"]), lse=_ptr(saved["lse"]), den=_ptr(saved["den"]))
+    st = load().sla_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), ctypes.byref(params), ctypes.byref(sv),
+                             _ptr(fwd_workspace), fwd_workspace.numel(), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dW),
+                             _ptr(dalpha), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "sla_backward")
+    return dq, dk, dv, (dalpha if sla2 else dW), workspace

@@ -864,6 +864,21 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 
     const float alpha = MODE == kModeSLA2 ? a.alpha[h] : 0.0f;
     const float inv_den = 1.0f / den;
+    // training forward: O^s, O^l, the row's log-normaliser and den, row by row
+    const int grow = blk * 64 + (tid & 63);
+    const bool srow = MODE != kModeDense && !QNT && a.save_os != nullptr && grow < N && (!isB || validB);
+    const size_t sidx = size_t(bh) * (size_t(Nb) * 64) + grow;
+    auto save_row = [&](__nv_bfloat16* dst, int ch, const float* v, float mul) {
+      uint4* p = reinterpret_cast<uint4*>(dst + sidx * D + ch * 32);
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8)
+        p[q8] = make_uint4(pack_bf16(v[8 * q8] * mul, v[8 * q8 + 1] * mul), pack_bf16(v[8 * q8 + 2] * mul, v[8 * q8 + 3] * mul),
+                           pack_bf16(v[8 * q8 + 4] * mul, v[8 * q8 + 5] * mul), pack_bf16(v[8 * q8 + 6] * mul, v[8 * q8 + 7] * mul));
+    };
+    if (srow) {
+      a.save_lse[sidx] = (m + log2f(l)) * 0.69314718055994531f;
+      a.save_den[sidx] = has_marg ? den : 0.0f;
+    }
     // O is staged as a bf16 pair tile in the P region (free after the last PV)
     // and written by TMA; the tensor map's row extent N drops the pad rows
     unsigned char* Ot = smem + C::oP;
@@ -875,6 +890,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         float nm[32];
         tmem_ld32(tq + (isB ? C::cNumB : C::cNumA) + ch * 32, nm);
         tmem_wait_ld();
+        if (srow) save_row(a.save_ol, ch, nm, inv_den);
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           const int e0 = ch * 32 + q8 * 8;
@@ -905,6 +921,15 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         const float os = o[i] * inv_l;
         const float ol = use_y ? x[i] : (has_marg ? x[i] * inv_den : 0.0f);
         out[i] = MODE == kModeSLA2 ? alpha * os + (1.0f - alpha) * ol : os + ol;
+      }
+      if (srow) {
+        save_row(a.save_os, ch, o, inv_l);
+        if (!use_y && has_marg) save_row(a.save_ol, ch, x, inv_den);
+        if (!has_marg) {  // no marginal block: O^l = 0 (x was never loaded)
+          uint4* p = reinterpret_cast<uint4*>(a.save_ol + sidx * D + ch * 32);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) p[q8] = make_uint4(0, 0, 0, 0);
+        }
       }
 #pragma unroll
       for (int q8 = 0; q8 < 4; ++q8) {

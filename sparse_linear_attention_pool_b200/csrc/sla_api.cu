@@ -72,8 +72,12 @@ size_t sla_workspace_size(const sla_params* p) {
   return make_layout(*p).total;
 }
 
-sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, const sla_params* p,
-                       void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+sla_status run_forward(const void* Q, const void* K, const void* V, void* O, const sla_params* p,
+                       void* workspace, size_t workspace_bytes, void* stream, const sla_saved* saved) {
   sla_status st = check_params(p);
   if (st != SLA_OK) return st;
   if (!Q || !K || !V || !O) return SLA_ERR_INVALID_ARG;
@@ -163,9 +167,113 @@ sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, con
     a.kn = L.kn;
     const float scale = p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / sqrtf(float(p->d));
     a.scale_log2 = scale * 1.4426950408889634f;
+    if (saved != nullptr) {
+      a.save_os = static_cast<__nv_bfloat16*>(saved->o_s);
+      a.save_ol = static_cast<__nv_bfloat16*>(saved->o_l);
+      a.save_lse = saved->lse;
+      a.save_den = saved->den;
+    }
     e = launch_attention(a, L.BH, L.d, sla2 ? kModeSLA2 : kModeSLA, s);
   }
   mark(6);
+  return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
+}
+
+bool saved_ok(const sla_saved* sv) {
+  return sv != nullptr && sv->o_s && sv->o_l && sv->lse && sv->den && aligned(sv->o_s, 16) && aligned(sv->o_l, 16) &&
+         aligned(sv->lse, 4) && aligned(sv->den, 4);
+}
+
+}  // namespace
+
+extern "C" {
+
+sla_status sla_forward(const void* Q, const void* K, const void* V, void* O, const sla_params* p,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  return run_forward(Q, K, V, O, p, workspace, workspace_bytes, stream, nullptr);
+}
+
+sla_status sla_forward_train(const void* Q, const void* K, const void* V, void* O, const sla_params* p,
+                             const sla_saved* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  sla_status st = check_params(p);
+  if (st != SLA_OK) return st;
+  if (p->precision != SLA_PREC_BF16) return SLA_ERR_UNSUPPORTED;
+  if (saved == nullptr || !saved->o_s || !saved->o_l || !saved->lse || !saved->den) return SLA_ERR_INVALID_ARG;
+  if (!saved_ok(saved)) return SLA_ERR_ALIGNMENT;
+  return run_forward(Q, K, V, O, p, workspace, workspace_bytes, stream, saved);
+}
+
+size_t sla_backward_workspace_size(const sla_params* p) {
+  if (check_params(p) != SLA_OK) return 0;
+  return make_bw_layout(*p).total;
+}
+
+sla_status sla_backward(const void* Q, const void* K, const void* V, const void* dO, const sla_params* p,
+                        const sla_saved* saved, const void* fwd_workspace, size_t fwd_workspace_bytes, void* dQ,
+                        void* dK, void* dV, float* dW, float* dalpha, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  sla_status st = check_params(p);
+  if (st != SLA_OK) return st;
+  if (p->precision != SLA_PREC_BF16) return SLA_ERR_UNSUPPORTED;
+  const bool sla2 = p->variant == SLA_VARIANT_SLA2;
+  if (!Q || !K || !V || !dO || !dQ || !dK || !dV || saved == nullptr) return SLA_ERR_INVALID_ARG;
+  if (!saved->o_s || !saved->o_l || !saved->lse || !saved->den) return SLA_ERR_INVALID_ARG;
+  if ((dW != nullptr && sla2) || (dalpha != nullptr && !sla2)) return SLA_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(dO, 16) || !aligned(dQ, 16) ||
+      !aligned(dK, 16) || !aligned(dV, 16) || !saved_ok(saved) || (dW && !aligned(dW, 4)) ||
+      (dalpha && !aligned(dalpha, 4)) || (p->w_proj && !aligned(p->w_proj, 16)))
+    return SLA_ERR_ALIGNMENT;
+  const Layout L = make_layout(*p);
+  const BwLayout BL = make_bw_layout(*p);
+  if (fwd_workspace == nullptr || !aligned(fwd_workspace, 256) || fwd_workspace_bytes < L.total)
+    return SLA_ERR_WORKSPACE;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < BL.total) return SLA_ERR_WORKSPACE;
+  const unsigned char* fw = static_cast<const unsigned char*>(fwd_workspace);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  auto bf = [](const void* x) { return static_cast<const __nv_bfloat16*>(x); };
+  BwdArgs a{};
+  a.L = BL;
+  a.Q = bf(Q);
+  a.K = bf(K);
+  a.V = bf(V);
+  a.dO = bf(dO);
+  a.save_os = bf(saved->o_s);
+  a.save_ol = bf(saved->o_l);
+  a.save_lse = saved->lse;
+  a.save_den = saved->den;
+  a.w_proj = sla2 ? nullptr : bf(p->w_proj);
+  a.alpha = sla2 ? p->alpha : nullptr;
+  a.phik = reinterpret_cast<const __nv_bfloat16*>(fw + L.phik);
+  a.htot = reinterpret_cast<const float*>(fw + L.htot32);
+  a.ztot = reinterpret_cast<const float*>(fw + L.ztot);
+  a.zblk = reinterpret_cast<const float*>(fw + L.zblk);
+  a.mc = reinterpret_cast<const int8_t*>(fw + L.mc);
+  a.crit = reinterpret_cast<const int32_t*>(fw + L.crit);
+  a.neg = reinterpret_cast<const int32_t*>(fw + L.neg);
+  a.dnum = reinterpret_cast<__nv_bfloat16*>(ws + BL.dnum);
+  a.phiq = reinterpret_cast<__nv_bfloat16*>(ws + BL.phiq);
+  a.Drow = reinterpret_cast<float*>(ws + BL.drow);
+  a.dden = reinterpret_cast<float*>(ws + BL.dden);
+  a.dzblk = reinterpret_cast<float*>(ws + BL.dzblk);
+  a.dztot = reinterpret_cast<float*>(ws + BL.dztot);
+  a.hblk = reinterpret_cast<float*>(ws + BL.hblk);
+  a.dhblk = reinterpret_cast<float*>(ws + BL.dhblk);
+  a.dhtot = reinterpret_cast<float*>(ws + BL.dhtot);
+  a.dwpart = reinterpret_cast<float*>(ws + BL.dwpart);
+  a.dapart = reinterpret_cast<float*>(ws + BL.dapart);
+  a.colC = reinterpret_cast<int*>(ws + BL.colc);
+  a.colE = reinterpret_cast<int*>(ws + BL.cole);
+  a.cntC = reinterpret_cast<int*>(ws + BL.cntc);
+  a.cntE = reinterpret_cast<int*>(ws + BL.cnte);
+  a.dQ = static_cast<__nv_bfloat16*>(dQ);
+  a.dK = static_cast<__nv_bfloat16*>(dK);
+  a.dV = static_cast<__nv_bfloat16*>(dV);
+  a.dW = sla2 ? nullptr : dW;
+  a.dalpha = sla2 ? dalpha : nullptr;
+  a.scale = p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / sqrtf(float(p->d));
+  a.sla = !sla2;
+  a.phi_elu1 = p->phi == SLA_PHI_ELU1 ? 1 : 0;
+  const cudaError_t e = launch_backward(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
 }
 

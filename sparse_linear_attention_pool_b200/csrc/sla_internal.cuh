@@ -133,9 +133,77 @@ struct AttnArgs {
   const float* vscale;         // [BH, Nb]
   int H, N, Nb, kc, kn;
   float scale_log2;            // softmax scale * log2(e)
+  // training forward (bf16 only; null otherwise): what the backward reads
+  __nv_bfloat16* save_os;      // [BH, Npad, d] O^s
+  __nv_bfloat16* save_ol;      // [BH, Npad, d] O^l (before SLA's W)
+  float* save_lse;             // [BH, Npad] log sum exp(scale q.k) over the critical keys
+  float* save_den;             // [BH, Npad] phi(q) . Z_i (0 without a marginal block)
 };
 enum AttnMode { kModeSLA = 0, kModeSLA2 = 1, kModeDense = 2 };
 cudaError_t launch_attention(const AttnArgs& a, int BH, int d, int mode, cudaStream_t s);
+
+// Backward workspace: per-row and per-block intermediates of the gradient.
+struct BwLayout {
+  int B, H, BH, N, Npad, Nb, d, kc, kn;
+  bool linear, sla;
+  size_t dnum, phiq, drow, dden, dzblk, dztot, hblk, dhblk, dhtot, dwpart, dapart, colc, cole, cntc, cnte, total;
+};
+
+inline BwLayout make_bw_layout(const sla_params& p) {
+  BwLayout L{};
+  L.B = p.B;
+  L.H = p.H;
+  L.BH = p.B * p.H;
+  L.N = p.N;
+  L.Nb = (p.N + kBlock - 1) / kBlock;
+  L.Npad = L.Nb * kBlock;
+  L.d = p.d;
+  L.kc = p.k_crit;
+  L.kn = p.k_neg;
+  L.linear = L.kc + L.kn < L.Nb;
+  L.sla = p.variant == SLA_VARIANT_SLA;
+  const size_t BH = size_t(L.BH), Nb = size_t(L.Nb), d = size_t(L.d), rows = BH * size_t(L.Npad);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.dnum = take(rows * d * 2);               // bf16 dO^l / den
+  L.phiq = take(rows * d * 2);               // bf16 phi(Q)
+  L.drow = take(rows * 4);                   // dO^s . O^s
+  L.dden = take(rows * 4);                   // -(dO^l . O^l) / den
+  L.dzblk = take(BH * Nb * d * 4);           // dZ_i
+  L.dztot = take(BH * d * 4);
+  L.hblk = take(L.linear ? BH * Nb * d * d * 4 : 0);   // h_j
+  L.dhblk = take(L.linear ? BH * Nb * d * d * 4 : 0);  // dH_i
+  L.dhtot = take(BH * d * d * 4);
+  L.dwpart = take(L.sla ? BH * Nb * d * d * 4 : 0);    // per-block O^l^T dO
+  L.dapart = take(BH * Nb * 4);                        // per-block dO . (O^s - O^l), [H][B][Nb]
+  L.colc = take(BH * Nb * Nb * 4);
+  L.cole = take(BH * Nb * Nb * 4);
+  L.cntc = take(BH * Nb * 4);
+  L.cnte = take(BH * Nb * 4);
+  L.total = off;
+  return L;
+}
+
+struct BwdArgs {
+  BwLayout L;
+  const __nv_bfloat16 *Q, *K, *V, *dO, *save_os, *save_ol, *w_proj, *phik;
+  const float *save_lse, *save_den, *alpha, *htot, *ztot, *zblk;
+  const int8_t* mc;
+  const int32_t *crit, *neg;
+  __nv_bfloat16 *dnum, *phiq;
+  float *Drow, *dden, *dzblk, *dztot, *hblk, *dhblk, *dhtot, *dwpart, *dapart;
+  int *colC, *colE, *cntC, *cntE;
+  __nv_bfloat16 *dQ, *dK, *dV;
+  float *dW, *dalpha;
+  float scale;
+  bool sla;
+  int phi_elu1;
+};
+cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s);
 
 // ---- device helpers ----
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }

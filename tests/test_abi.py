@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sla_abi_version() == 3
+    assert lib.sla_abi_version() == 4
     for s in range(8):
         assert sla.status_string(s)
     assert "unknown" in sla.status_string(99)

@@ -32,7 +32,7 @@ import numpy as np
 BLOCK = 64  # bq = bkv = 64 tokens per block
 
 # stream ids for SeedSequence spawn keys
-_T_Q, _T_K, _T_V, _T_WPROJ, _T_PROJQ, _T_PROJK, _T_ALPHA = range(7)
+_T_Q, _T_K, _T_V, _T_WPROJ, _T_PROJQ, _T_PROJK, _T_ALPHA, _T_DO = range(8)
 
 # value written into the rows past N of a padded tensor; a kernel that reads
 # them by mistake produces visibly wrong results
@@ -178,6 +178,26 @@ def head_tensor(w: Workload, tensor: str, b: int, h: int) -> np.ndarray:
     if Np > w.N:
         x[w.N:] = np.float32(w.pad_value)
     return f32_to_bf16_bits(x)
+
+
+def head_grad_output(w: Workload, b: int, h: int) -> np.ndarray:
+    """Upstream gradient dO of one head for the backward pass: N(0, 1), bf16
+    bits [N_pad, d]; rows >= N hold pad_value (the backward must ignore them)."""
+    rng = _rng(w.seed, _T_DO, b, h)
+    x = rng.standard_normal((w.N_pad, w.d), dtype=np.float32)
+    if w.N_pad > w.N:
+        x[w.N:] = np.float32(w.pad_value)
+    return f32_to_bf16_bits(x)
+
+
+def grad_output(w: Workload, heads: Optional[Iterable[tuple[int, int]]] = None) -> np.ndarray:
+    """dO for every head ([B, H, N_pad, d]) or for a list of heads ([len, 1, N_pad, d])."""
+    full = heads is None
+    hl = [(b, h) for b in range(w.B) for h in range(w.H)] if full else list(heads)
+    out = np.empty(((w.B, w.H) if full else (len(hl), 1)) + (w.N_pad, w.d), dtype=np.uint16)
+    for idx, (b, h) in enumerate(hl):
+        out[(b, h) if full else (idx, 0)] = head_grad_output(w, b, h)
+    return out
 
 
 def weight(w: Workload, which: str) -> np.ndarray:
