@@ -413,6 +413,45 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(const PrepArgs a) {
   }
 }
 
+// dst (bf16 [D][LD] tile) = tot - sum over the listed blocks of blk[j] (fp32
+// d x d each), and zdst[c] = ztot[c] - sum of zblk[j][c]: the complement sums
+// of H_i, Z_i (query side) and A_j, b_j (key side). Each thread keeps its
+// D * D / 128 entries in registers and subtracts block after block (coalesced
+// float4 loads, independent across the thread's entries), in list order.
+template <int D>
+__device__ __forceinline__ void complement_sum(bf16* dst, float* zdst, const float* tot, const float* blk,
+                                               const float* ztot, const float* zblk, const int32_t* l1, int n1,
+                                               const int32_t* l2, int n2) {
+  constexpr int PER = D * D / 4 / 128;
+  const int tid = threadIdx.x;
+  float4 acc[PER];
+  const float4* t4 = reinterpret_cast<const float4*>(tot);
+#pragma unroll
+  for (int k = 0; k < PER; ++k) acc[k] = t4[tid + 128 * k];
+  float z = tid < D ? ztot[tid] : 0.0f;
+  auto sub = [&](int j) {
+    const float4* b4 = reinterpret_cast<const float4*>(blk + size_t(j) * D * D);
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const float4 v = b4[tid + 128 * k];
+      acc[k].x -= v.x;
+      acc[k].y -= v.y;
+      acc[k].z -= v.z;
+      acc[k].w -= v.w;
+    }
+    if (tid < D) z -= zblk[size_t(j) * D + tid];
+  };
+  for (int u = 0; u < n1; ++u) sub(l1[u]);
+  for (int u = 0; u < n2; ++u) sub(l2[u]);
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int e = 4 * (tid + 128 * k), r = e / D, c = e % D;
+    *reinterpret_cast<uint2*>(dst + r * Bw<D>::LD + c) =
+        make_uint2(pack_bf16(acc[k].x, acc[k].y), pack_bf16(acc[k].z, acc[k].w));
+  }
+  if (tid < D) zdst[tid] = z;
+}
+
 // ---------------------------------------------------------------------------
 // dQ per query block: the sparse pairs, then the linear branch
 // ---------------------------------------------------------------------------
@@ -433,20 +472,38 @@ __global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   bf16* Qs = reinterpret_cast<bf16*>(smem_raw);
   bf16* dOs = Qs + T::kTile;
-  bf16* Ks = dOs + T::kTile;
-  bf16* Vs = Ks + T::kTile;
-  bf16* Hs = Vs + T::kTile;    // [D][LD]: H_i
-  bf16* dns = Hs + T::kMat;    // dnum tile
-  float* zis = reinterpret_cast<float*>(dns + T::kTile);  // [D]: Z_i
+  bf16* dns = dOs + T::kTile;  // dnum tile
+  bf16* KVs = dns + T::kTile;  // [2 buffers][K tile, V tile]
+  bf16* Hs = KVs + 4 * T::kTile;  // [D][LD]: H_i
+  float* zis = reinterpret_cast<float*>(Hs + T::kMat);  // [D]: Z_i
   const int i = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
   const int t0 = i * 64, nv = min(64, a.N - t0);
   const float asc = a.alpha ? a.alpha[bh % a.H] : 1.0f;  // dO^s = asc dO
+  const bool linear = a.kc + a.kn < a.Nb;
   const size_t rowbase = size_t(bh) * a.Npad + t0;
   const size_t headbase = size_t(bh) * a.Npad * D;
+  const int32_t* crit = a.crit + (size_t(bh) * a.Nb + i) * a.kc;
   load_tile<D>(Qs, a.Q + rowbase * D, nv);
   load_tile<D>(dOs, a.dO + rowbase * D, nv);
+  if (linear) load_tile<D>(dns, a.dnum + rowbase * D, nv);
   cp_async_commit();
+  auto load_pair = [&](int t) {
+    const int j = crit[t];
+    const int nvj = min(64, a.N - j * 64);
+    bf16* buf = KVs + (t & 1) * 2 * T::kTile;
+    load_tile<D>(buf, a.K + headbase + size_t(j) * 64 * D, nvj);
+    load_tile<D>(buf + T::kTile, a.V + headbase + size_t(j) * 64 * D, nvj);
+    cp_async_commit();
+  };
+  load_pair(0);
+  // H_i = H_tot - sum over the excluded blocks of h_j, Z_i likewise (while the
+  // first tiles land)
+  if (linear)
+    complement_sum<D>(Hs, zis, a.htot + size_t(bh) * D * D, a.hblk + size_t(bh) * a.Nb * D * D,
+                      a.ztot + size_t(bh) * D, a.zblk + size_t(bh) * a.Nb * D, crit, a.kc,
+                      a.neg + (size_t(bh) * a.Nb + i) * a.kn, a.kn);
+
   const int r0 = warp * 16, ra = r0 + g, rb = ra + 8;
   const bool va = ra < nv, vb = rb < nv;
   const float lse2a = va ? a.lse[rowbase + ra] * kLog2e : INFINITY;
@@ -456,16 +513,17 @@ __global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
   float dq[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) dq[nt][0] = dq[nt][1] = dq[nt][2] = dq[nt][3] = 0.0f;
-  const int32_t* crit = a.crit + (size_t(bh) * a.Nb + i) * a.kc;
   for (int t = 0; t < a.kc; ++t) {
-    const int j = crit[t];
-    const int nvj = min(64, a.N - j * 64);
-    __syncthreads();  // the previous pair's K / V reads are done
-    load_tile<D>(Ks, a.K + headbase + size_t(j) * 64 * D, nvj);
-    load_tile<D>(Vs, a.V + headbase + size_t(j) * 64 * D, nvj);
-    cp_async_commit();
-    cp_async_wait<0>();
+    if (t + 1 < a.kc) {
+      load_pair(t + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
+    const bf16* Ks = KVs + (t & 1) * 2 * T::kTile;
+    const bf16* Vs = Ks + T::kTile;
+    const int nvj = min(64, a.N - crit[t] * 64);
     float s[8][4], dp[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
@@ -482,35 +540,15 @@ __global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
         s[nt][e] = p * (asc * dp[nt][e] - (e < 2 ? Da : Db));  // dS
       }
     mma_pz<NT>(dq, s, Ks, T::LD, g, q);
+    __syncthreads();  // this buffer is refilled two pairs on
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dq[nt][e] *= a.scale;
 
-  if (a.kc + a.kn < a.Nb) {
-    // H_i = H_tot - sum over the excluded blocks of h_j (bf16), Z_i likewise
-    __syncthreads();
-    const int32_t* neg = a.neg + (size_t(bh) * a.Nb + i) * a.kn;
-    const float* ht = a.htot + size_t(bh) * D * D;
-    const float* hb = a.hblk + size_t(bh) * a.Nb * D * D;
-    for (int e = threadIdx.x; e < D * D; e += 128) {
-      float v = ht[e];
-      for (int u = 0; u < a.kc; ++u) v -= hb[size_t(crit[u]) * D * D + e];
-      for (int u = 0; u < a.kn; ++u) v -= hb[size_t(neg[u]) * D * D + e];
-      Hs[(e / D) * T::LD + (e % D)] = __float2bfloat16_rn(v);
-    }
-    for (int c = threadIdx.x; c < D; c += 128) {
-      float v = a.ztot[size_t(bh) * D + c];
-      for (int u = 0; u < a.kc; ++u) v -= a.zblk[(size_t(bh) * a.Nb + crit[u]) * D + c];
-      for (int u = 0; u < a.kn; ++u) v -= a.zblk[(size_t(bh) * a.Nb + neg[u]) * D + c];
-      zis[c] = v;
-    }
-    load_tile<D>(dns, a.dnum + rowbase * D, nv);
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    // dphi(Q_i) = dnum H_i^T + dden Z_i^T
+  if (linear) {
+    // dphi(Q_i) = dnum H_i^T + dden Z_i^T, through the feature map's Jacobian
     float u[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) u[nt][0] = u[nt][1] = u[nt][2] = u[nt][3] = 0.0f;
@@ -558,12 +596,11 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
   bf16* Ks = reinterpret_cast<bf16*>(smem_raw);
   bf16* Vs = Ks + T::kTile;
   bf16* PKs = Vs + T::kTile;
-  bf16* Qs = PKs + T::kTile;
-  bf16* dOs = Qs + T::kTile;
-  bf16* As = dOs + T::kTile;  // [D][LD]: A_j
+  bf16* QOs = PKs + T::kTile;     // [2 buffers][Q tile, dO tile]
+  bf16* As = QOs + 4 * T::kTile;  // [D][LD]: A_j
   float* bjs = reinterpret_cast<float*>(As + T::kMat);  // [D]
-  float* lse2s = bjs + D;                               // [64]
-  float* Ds = lse2s + 64;                               // [64]
+  float* lse2s = bjs + D;                               // [2][64]
+  float* Ds = lse2s + 128;                              // [2][64]
   const int j = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
   const int t0 = j * 64, nvj = min(64, a.N - t0);
@@ -574,6 +611,30 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
   load_tile<D>(Vs, a.V + rowbase * D, nvj);
   load_tile<D>(PKs, a.phik + rowbase * D, nvj);
   cp_async_commit();
+  const int nC = a.cntC[size_t(bh) * a.Nb + j];
+  const int* colC = a.colC + (size_t(bh) * a.Nb + j) * a.Nb;
+  auto load_pair = [&](int t) {
+    const int i = colC[t];
+    const int nvi = min(64, a.N - i * 64);
+    const int b = t & 1;
+    bf16* buf = QOs + b * 2 * T::kTile;
+    load_tile<D>(buf, a.Q + (headrow + size_t(i) * 64) * D, nvi);
+    load_tile<D>(buf + T::kTile, a.dO + (headrow + size_t(i) * 64) * D, nvi);
+    cp_async_commit();
+    if (threadIdx.x < 64) {
+      const int r = threadIdx.x;
+      lse2s[b * 64 + r] = r < nvi ? a.lse[headrow + i * 64 + r] * kLog2e : INFINITY;
+      Ds[b * 64 + r] = r < nvi ? a.Drow[headrow + i * 64 + r] : 0.0f;
+    }
+  };
+  if (nC > 0) load_pair(0);
+  // A_j = dH_tot - sum over the query blocks that exclude j of dH_i, b_j likewise
+  if (a.linear) {
+    const int nE = a.cntE[size_t(bh) * a.Nb + j];
+    complement_sum<D>(As, bjs, a.dhtot + size_t(bh) * D * D, a.dhblk + size_t(bh) * a.Nb * D * D,
+                      a.dztot + size_t(bh) * D, a.dzblk + size_t(bh) * a.Nb * D,
+                      a.colE + (size_t(bh) * a.Nb + j) * a.Nb, nE, nullptr, 0);
+  }
   const int r0 = warp * 16, ra = r0 + g, rb = ra + 8;
   const bool va = ra < nvj, vb = rb < nvj;
 
@@ -582,22 +643,18 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[nt][e] = dv[nt][e] = 0.0f;
-  const int nC = a.cntC[size_t(bh) * a.Nb + j];
-  const int* colC = a.colC + (size_t(bh) * a.Nb + j) * a.Nb;
   for (int t = 0; t < nC; ++t) {
-    const int i = colC[t];
-    const int nvi = min(64, a.N - i * 64);
-    __syncthreads();  // the previous pair's Q / dO reads are done
-    load_tile<D>(Qs, a.Q + (headrow + size_t(i) * 64) * D, nvi);
-    load_tile<D>(dOs, a.dO + (headrow + size_t(i) * 64) * D, nvi);
-    cp_async_commit();
-    if (threadIdx.x < 64) {
-      const int r = threadIdx.x;
-      lse2s[r] = r < nvi ? a.lse[headrow + i * 64 + r] * kLog2e : INFINITY;
-      Ds[r] = r < nvi ? a.Drow[headrow + i * 64 + r] : 0.0f;
+    if (t + 1 < nC) {
+      load_pair(t + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    cp_async_wait<0>();
     __syncthreads();
+    const bf16* Qs = QOs + (t & 1) * 2 * T::kTile;
+    const bf16* dOs = Qs + T::kTile;
+    const float* l2 = lse2s + (t & 1) * 64;
+    const float* Dc = Ds + (t & 1) * 64;
     float st[8][4], dpt[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
@@ -610,7 +667,7 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
       for (int e = 0; e < 4; ++e) {
         const int col = nt * 8 + 2 * q + (e & 1);
         const bool vk = e < 2 ? va : vb;
-        st[nt][e] = vk ? ex2_approx(fmaf(st[nt][e], a.scale_log2, -lse2s[col])) : 0.0f;  // P^T
+        st[nt][e] = vk ? ex2_approx(fmaf(st[nt][e], a.scale_log2, -l2[col])) : 0.0f;  // P^T
       }
     mma_pz<NT>(dv, st, dOs, T::LD, g, q);                 // dV += P^T dO_i
     mma_xyt<8, D>(dpt, Vs, T::LD, r0, dOs, T::LD, g, q);  // dP^T = V_j dO_i^T
@@ -619,10 +676,13 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int col = nt * 8 + 2 * q + (e & 1);
-        st[nt][e] *= asc * dpt[nt][e] - Ds[col];  // dS^T
+        st[nt][e] *= asc * dpt[nt][e] - Dc[col];  // dS^T
       }
     mma_pz<NT>(dk, st, Qs, T::LD, g, q);  // dK += dS^T Q_i
+    __syncthreads();  // this buffer is refilled two pairs on
   }
+  cp_async_wait<0>();
+  __syncthreads();  // K, V, phi(K) and A_j are in place even without a sparse pair
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -632,24 +692,6 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
     }
 
   if (a.linear) {
-    // A_j = dH_tot - sum over the query blocks that exclude j of dH_i (bf16), b_j likewise
-    __syncthreads();
-    const int nE = a.cntE[size_t(bh) * a.Nb + j];
-    const int* colE = a.colE + (size_t(bh) * a.Nb + j) * a.Nb;
-    const float* dht = a.dhtot + size_t(bh) * D * D;
-    const float* dhb = a.dhblk + size_t(bh) * a.Nb * D * D;
-    for (int e = threadIdx.x; e < D * D; e += 128) {
-      float v = dht[e];
-      for (int u = 0; u < nE; ++u) v -= dhb[size_t(colE[u]) * D * D + e];
-      As[(e / D) * T::LD + (e % D)] = __float2bfloat16_rn(v);
-    }
-    for (int c = threadIdx.x; c < D; c += 128) {
-      float v = a.dztot[size_t(bh) * D + c];
-      for (int u = 0; u < nE; ++u) v -= a.dzblk[(size_t(bh) * a.Nb + colE[u]) * D + c];
-      bjs[c] = v;
-    }
-    cp_async_wait<0>();
-    __syncthreads();
     mma_xz<NT, D>(dv, PKs, T::LD, r0, As, T::LD, g, q);  // dV += phi(K_j) A_j
     store_frag_rows<NT>(a.dV + rowbase * D, D, ra, va, vb, dv, q);
     float u[NT][4];
@@ -673,7 +715,6 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) dk[nt][e] += u[nt][e];
   } else {
-    cp_async_wait<0>();
     store_frag_rows<NT>(a.dV + rowbase * D, D, ra, va, vb, dv, q);
   }
   store_frag_rows<NT>(a.dK + rowbase * D, D, ra, va, vb, dk, q);
@@ -735,7 +776,7 @@ cudaError_t run_backward(const BwdArgs& a, cudaStream_t s) {
   if (e == cudaSuccess) {
     QArgs qa{a.Q, a.K, a.V, a.dO, a.dnum, a.crit, a.neg, a.save_lse, a.Drow, a.dden, a.htot, a.hblk, a.ztot,
              a.zblk, alpha, a.dQ, scale, scale * kLog2e, L.H, L.N, L.Npad, Nb, L.kc, L.kn, a.phi_elu1};
-    const int bytes = (5 * T::kTile + T::kMat) * 2 + D * 4;
+    const int bytes = (7 * T::kTile + T::kMat) * 2 + D * 4;
     e = set_smem(bwd_q_kernel<D>, bytes);
     if (e == cudaSuccess) {
       bwd_q_kernel<D><<<blocks, 128, bytes, s>>>(qa);
@@ -747,7 +788,7 @@ cudaError_t run_backward(const BwdArgs& a, cudaStream_t s) {
     KVArgs ka{a.Q, a.K, a.V, a.dO, a.phik, a.colC, a.colE, a.cntC, a.cntE, a.save_lse, a.Drow, a.dhtot,
               a.dhblk, a.dztot, a.dzblk, alpha, a.dK, a.dV, scale, scale * kLog2e, L.H, L.N, L.Npad, Nb,
               L.linear ? 1 : 0, a.phi_elu1};
-    const int bytes = (5 * T::kTile + T::kMat) * 2 + (D + 128) * 4;
+    const int bytes = (7 * T::kTile + T::kMat) * 2 + (D + 256) * 4;
     e = set_smem(bwd_kv_kernel<D>, bytes);
     if (e == cudaSuccess) {
       bwd_kv_kernel<D><<<blocks, 128, bytes, s>>>(ka);
