@@ -62,37 +62,58 @@ __device__ __forceinline__ void load_tile(bf16* dst, const bf16* src, int nvalid
   }
 }
 
+// Fragments by ldmatrix from padded row-major tiles (row addresses 16-byte
+// aligned: the row stride is 2 (D + 8) = 16 (D / 8 + 1) bytes).
+// A: rows r0 .. r0+15, columns k0 .. k0+15
+__device__ __forceinline__ void lda(uint32_t* a, const bf16* X, int ldx, int r0, int k0, int lane) {
+  const int r = r0 + (lane & 7) + ((lane >> 3) & 1) * 8, c = k0 + (lane >> 4) * 8;
+  ldsm_x4(smem_u32(X + r * ldx + c), a[0], a[1], a[2], a[3]);
+}
+// B of n tiles n0 and n0 + 8 when B[k][n] = Y[n][k] (Y rows n, k contiguous):
+// b[0], b[1] for n0, b[2], b[3] for n0 + 8
+__device__ __forceinline__ void ldb_rows(uint32_t* b, const bf16* Y, int ldy, int n0, int k0, int lane) {
+  const int r = n0 + (lane & 7) + (lane >> 4) * 8, c = k0 + ((lane >> 3) & 1) * 8;
+  ldsm_x4(smem_u32(Y + r * ldy + c), b[0], b[1], b[2], b[3]);
+}
+// B of n tiles n0 and n0 + 8 when B[k][n] = Z[k][n] (Z rows k, n contiguous)
+__device__ __forceinline__ void ldb_cols(uint32_t* b, const bf16* Z, int ldz, int k0, int n0, int lane) {
+  const int r = k0 + (lane & 7) + ((lane >> 3) & 1) * 8, c = n0 + (lane >> 4) * 8;
+  ldsm_x4_t(smem_u32(Z + r * ldz + c), b[0], b[1], b[2], b[3]);
+}
+
 // acc[16 x 8 NTN] += X[r0 .. r0+15][0 .. K) * Y[0 .. 8 NTN)[0 .. K)^T
 template <int NTN, int K>
 __device__ __forceinline__ void mma_xyt(float (*acc)[4], const bf16* X, int ldx, int r0, const bf16* Y, int ldy,
-                                        int g, int q) {
+                                        int lane) {
 #pragma unroll
   for (int k0 = 0; k0 < K; k0 += 16) {
     uint32_t a[4];
-    a[0] = pair_row(X, ldx, r0 + g, k0 + 2 * q);
-    a[1] = pair_row(X, ldx, r0 + g + 8, k0 + 2 * q);
-    a[2] = pair_row(X, ldx, r0 + g, k0 + 8 + 2 * q);
-    a[3] = pair_row(X, ldx, r0 + g + 8, k0 + 8 + 2 * q);
+    lda(a, X, ldx, r0, k0, lane);
 #pragma unroll
-    for (int nt = 0; nt < NTN; ++nt)
-      mma16816(acc[nt], a, pair_row(Y, ldy, nt * 8 + g, k0 + 2 * q), pair_row(Y, ldy, nt * 8 + g, k0 + 8 + 2 * q));
+    for (int nt = 0; nt < NTN; nt += 2) {
+      uint32_t b[4];
+      ldb_rows(b, Y, ldy, nt * 8, k0, lane);
+      mma16816(acc[nt], a, b[0], b[1]);
+      mma16816(acc[nt + 1], a, b[2], b[3]);
+    }
   }
 }
 
 // acc[16 x 8 NTN] += X[r0 .. r0+15][0 .. K) * Z[0 .. K)[0 .. 8 NTN)
 template <int NTN, int K>
 __device__ __forceinline__ void mma_xz(float (*acc)[4], const bf16* X, int ldx, int r0, const bf16* Z, int ldz,
-                                       int g, int q) {
+                                       int lane) {
 #pragma unroll
   for (int k0 = 0; k0 < K; k0 += 16) {
     uint32_t a[4];
-    a[0] = pair_row(X, ldx, r0 + g, k0 + 2 * q);
-    a[1] = pair_row(X, ldx, r0 + g + 8, k0 + 2 * q);
-    a[2] = pair_row(X, ldx, r0 + g, k0 + 8 + 2 * q);
-    a[3] = pair_row(X, ldx, r0 + g + 8, k0 + 8 + 2 * q);
+    lda(a, X, ldx, r0, k0, lane);
 #pragma unroll
-    for (int nt = 0; nt < NTN; ++nt)
-      mma16816(acc[nt], a, pair_col(Z, ldz, k0 + 2 * q, nt * 8 + g), pair_col(Z, ldz, k0 + 8 + 2 * q, nt * 8 + g));
+    for (int nt = 0; nt < NTN; nt += 2) {
+      uint32_t b[4];
+      ldb_cols(b, Z, ldz, k0, nt * 8, lane);
+      mma16816(acc[nt], a, b[0], b[1]);
+      mma16816(acc[nt + 1], a, b[2], b[3]);
+    }
   }
 }
 
@@ -100,7 +121,7 @@ __device__ __forceinline__ void mma_xz(float (*acc)[4], const bf16* X, int ldx, 
 // fragments p[8][4] of an earlier product (the C layout of m16n8 is the A
 // layout of the next m16n8k16)
 template <int NTN>
-__device__ __forceinline__ void mma_pz(float (*acc)[4], const float (*p)[4], const bf16* Z, int ldz, int g, int q) {
+__device__ __forceinline__ void mma_pz(float (*acc)[4], const float (*p)[4], const bf16* Z, int ldz, int lane) {
 #pragma unroll
   for (int kt = 0; kt < 4; ++kt) {
     uint32_t a[4];
@@ -109,9 +130,12 @@ __device__ __forceinline__ void mma_pz(float (*acc)[4], const float (*p)[4], con
     a[2] = pack_bf16(p[2 * kt + 1][0], p[2 * kt + 1][1]);
     a[3] = pack_bf16(p[2 * kt + 1][2], p[2 * kt + 1][3]);
 #pragma unroll
-    for (int nt = 0; nt < NTN; ++nt)
-      mma16816(acc[nt], a, pair_col(Z, ldz, kt * 16 + 2 * q, nt * 8 + g),
-               pair_col(Z, ldz, kt * 16 + 8 + 2 * q, nt * 8 + g));
+    for (int nt = 0; nt < NTN; nt += 2) {
+      uint32_t b[4];
+      ldb_cols(b, Z, ldz, kt * 16, nt * 8, lane);
+      mma16816(acc[nt], a, b[0], b[1]);
+      mma16816(acc[nt + 1], a, b[2], b[3]);
+    }
   }
 }
 
@@ -325,7 +349,7 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(const PrepArgs a) {
   if (SLA && a.W != nullptr) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) u[nt][0] = u[nt][1] = u[nt][2] = u[nt][3] = 0.0f;
-    mma_xyt<NT, D>(u, dOs, T::LD, warp * 16, Ws, T::LD, g, q);
+    mma_xyt<NT, D>(u, dOs, T::LD, warp * 16, Ws, T::LD, lane);
   } else {  // SLA without W (identity) or SLA2
     frag_from_tile<NT>(u, dOs, T::LD, ra, g, q);
     const float lmul = SLA ? 1.0f : 1.0f - alpha;
@@ -529,8 +553,8 @@ __global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.0f;
-    mma_xyt<8, D>(s, Qs, T::LD, r0, Ks, T::LD, g, q);
-    mma_xyt<8, D>(dp, dOs, T::LD, r0, Vs, T::LD, g, q);
+    mma_xyt<8, D>(s, Qs, T::LD, r0, Ks, T::LD, lane);
+    mma_xyt<8, D>(dp, dOs, T::LD, r0, Vs, T::LD, lane);
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -539,7 +563,7 @@ __global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
         const float p = key < nvj ? ex2_approx(fmaf(s[nt][e], a.scale_log2, -(e < 2 ? lse2a : lse2b))) : 0.0f;
         s[nt][e] = p * (asc * dp[nt][e] - (e < 2 ? Da : Db));  // dS
       }
-    mma_pz<NT>(dq, s, Ks, T::LD, g, q);
+    mma_pz<NT>(dq, s, Ks, T::LD, lane);
     __syncthreads();  // this buffer is refilled two pairs on
   }
 #pragma unroll
@@ -552,7 +576,7 @@ __global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
     float u[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) u[nt][0] = u[nt][1] = u[nt][2] = u[nt][3] = 0.0f;
-    mma_xyt<NT, D>(u, dns, T::LD, r0, Hs, T::LD, g, q);
+    mma_xyt<NT, D>(u, dns, T::LD, r0, Hs, T::LD, lane);
     const float dda = va ? a.dden[rowbase + ra] : 0.0f, ddb = vb ? a.dden[rowbase + rb] : 0.0f;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -660,7 +684,7 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) st[nt][e] = dpt[nt][e] = 0.0f;
-    mma_xyt<8, D>(st, Ks, T::LD, r0, Qs, T::LD, g, q);  // S^T = K_j Q_i^T
+    mma_xyt<8, D>(st, Ks, T::LD, r0, Qs, T::LD, lane);  // S^T = K_j Q_i^T
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -669,8 +693,8 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
         const bool vk = e < 2 ? va : vb;
         st[nt][e] = vk ? ex2_approx(fmaf(st[nt][e], a.scale_log2, -l2[col])) : 0.0f;  // P^T
       }
-    mma_pz<NT>(dv, st, dOs, T::LD, g, q);                 // dV += P^T dO_i
-    mma_xyt<8, D>(dpt, Vs, T::LD, r0, dOs, T::LD, g, q);  // dP^T = V_j dO_i^T
+    mma_pz<NT>(dv, st, dOs, T::LD, lane);                 // dV += P^T dO_i
+    mma_xyt<8, D>(dpt, Vs, T::LD, r0, dOs, T::LD, lane);  // dP^T = V_j dO_i^T
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -678,7 +702,7 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
         const int col = nt * 8 + 2 * q + (e & 1);
         st[nt][e] *= asc * dpt[nt][e] - Dc[col];  // dS^T
       }
-    mma_pz<NT>(dk, st, Qs, T::LD, g, q);  // dK += dS^T Q_i
+    mma_pz<NT>(dk, st, Qs, T::LD, lane);  // dK += dS^T Q_i
     __syncthreads();  // this buffer is refilled two pairs on
   }
   cp_async_wait<0>();
@@ -692,12 +716,12 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
     }
 
   if (a.linear) {
-    mma_xz<NT, D>(dv, PKs, T::LD, r0, As, T::LD, g, q);  // dV += phi(K_j) A_j
+    mma_xz<NT, D>(dv, PKs, T::LD, r0, As, T::LD, lane);  // dV += phi(K_j) A_j
     store_frag_rows<NT>(a.dV + rowbase * D, D, ra, va, vb, dv, q);
     float u[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) u[nt][0] = u[nt][1] = u[nt][2] = u[nt][3] = 0.0f;
-    mma_xyt<NT, D>(u, Vs, T::LD, r0, As, T::LD, g, q);  // V_j A_j^T
+    mma_xyt<NT, D>(u, Vs, T::LD, r0, As, T::LD, lane);  // V_j A_j^T
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int c = nt * 8 + 2 * q;
