@@ -346,7 +346,7 @@ def time_dense(sla, w, dev, steps, warmup):
 ROUTER_TAU = 1e-2
 
 
-def time_backward(sla, w, dev, steps, warmup):
+def time_backward(sla, w, dev, steps, warmup, dense=True):
     """(ms per sla_backward call, ms per sla_forward_train call, ms per dense
     FlashAttention backward of the same shape through torch's
     scaled_dot_product_attention, for context; None where unavailable)."""
@@ -374,6 +374,8 @@ def time_backward(sla, w, dev, steps, warmup):
                                      workspace=bws), steps, warmup)
     fwd = timed(lambda: sla.forward_train(dev["q"], dev["k"], dev["v"], params=p, out=out, workspace=fws,
                                           saved=saved), steps, warmup)
+    if not dense:
+        return bwd, fwd, None
     dense = None
     try:
         qd, kd, vd = (dev[x][:, :, :w.N].detach().clone().requires_grad_(True) for x in ("q", "k", "v"))
@@ -656,6 +658,24 @@ def run_sweep(args):
                       "dtype": "bf16"}), flush=True)
 
 
+def run_backward_only(args):
+    """The backward pass alone on one workload: one sla_forward_train, then
+    `warmup` + `steps` sla_backward calls and as many training forwards (mask
+    fixed, inputs resident). One JSON line; for profiling."""
+    import sparse_linear_attention_pool_b200 as sla
+
+    sla.load()
+    w = W.WORKLOADS[args.workload]
+    if w.precision != "bf16":
+        raise SystemExit("the backward pass is bf16 only")
+    dev = device_inputs(W.make_inputs(w))
+    bms, fms, dms = time_backward(sla, w, dev, args.steps, args.warmup, dense=not args.no_dense)
+    print(json.dumps({"workload": w.name, "steps": args.steps, "warmup": args.warmup,
+                      "backward_ms": round(bms, 4), "forward_train_ms": round(fms, 4),
+                      "backward_tflops": round(backward_flops(w) / (bms * 1e-3) / 1e12, 2),
+                      "dense_flash_backward_ms": None if dms is None else round(dms, 4)}), flush=True)
+
+
 def run_reference(args):
     """The oracle as it stands, timed on the host cores: one head per step."""
     rank = int(os.environ.get("RANK", "0"))
@@ -699,6 +719,8 @@ def main():
     ap.add_argument("--dense-steps", type=int, default=5)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time sla_backward alone on --workload (one JSON line)")
     ap.add_argument("--no-north-star", action="store_true")
     ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--sweep", action="store_true",
@@ -709,6 +731,8 @@ def main():
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.sweep:
         run_sweep(args)
+    elif args.backward_only:
+        run_backward_only(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -117,13 +117,13 @@ __device__ __forceinline__ void mma_xz(float (*acc)[4], const bf16* X, int ldx, 
   }
 }
 
-// acc[16 x 8 NTN] += P * Z[0 .. 64)[0 .. 8 NTN), P the 16 x 64 accumulator
-// fragments p[8][4] of an earlier product (the C layout of m16n8 is the A
-// layout of the next m16n8k16)
-template <int NTN>
+// acc[16 x 8 NTN] += P * Z[0 .. 16 KT)[0 .. 8 NTN), P the 16 x 16 KT
+// accumulator fragments p[2 KT][4] of an earlier product (the C layout of
+// m16n8 is the A layout of the next m16n8k16)
+template <int NTN, int KT>
 __device__ __forceinline__ void mma_pz(float (*acc)[4], const float (*p)[4], const bf16* Z, int ldz, int lane) {
 #pragma unroll
-  for (int kt = 0; kt < 4; ++kt) {
+  for (int kt = 0; kt < KT; ++kt) {
     uint32_t a[4];
     a[0] = pack_bf16(p[2 * kt][0], p[2 * kt][1]);
     a[1] = pack_bf16(p[2 * kt][2], p[2 * kt][3]);
@@ -439,25 +439,25 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(const PrepArgs a) {
 
 // dst (bf16 [D][LD] tile) = tot - sum over the listed blocks of blk[j] (fp32
 // d x d each), and zdst[c] = ztot[c] - sum of zblk[j][c]: the complement sums
-// of H_i, Z_i (query side) and A_j, b_j (key side). Each thread keeps its
-// D * D / 128 entries in registers and subtracts block after block (coalesced
+// of H_i, Z_i (query side) and A_j, b_j (key side). Each of the NTH threads
+// keeps its D * D / NTH entries in registers and subtracts block after block (coalesced
 // float4 loads, independent across the thread's entries), in list order.
-template <int D>
+template <int D, int NTH>
 __device__ __forceinline__ void complement_sum(bf16* dst, float* zdst, const float* tot, const float* blk,
                                                const float* ztot, const float* zblk, const int32_t* l1, int n1,
                                                const int32_t* l2, int n2) {
-  constexpr int PER = D * D / 4 / 128;
+  constexpr int PER = D * D / 4 / NTH;
   const int tid = threadIdx.x;
   float4 acc[PER];
   const float4* t4 = reinterpret_cast<const float4*>(tot);
 #pragma unroll
-  for (int k = 0; k < PER; ++k) acc[k] = t4[tid + 128 * k];
+  for (int k = 0; k < PER; ++k) acc[k] = t4[tid + NTH * k];
   float z = tid < D ? ztot[tid] : 0.0f;
   auto sub = [&](int j) {
     const float4* b4 = reinterpret_cast<const float4*>(blk + size_t(j) * D * D);
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
-      const float4 v = b4[tid + 128 * k];
+      const float4 v = b4[tid + NTH * k];
       acc[k].x -= v.x;
       acc[k].y -= v.y;
       acc[k].z -= v.z;
@@ -469,7 +469,7 @@ __device__ __forceinline__ void complement_sum(bf16* dst, float* zdst, const flo
   for (int u = 0; u < n2; ++u) sub(l2[u]);
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
-    const int e = 4 * (tid + 128 * k), r = e / D, c = e % D;
+    const int e = 4 * (tid + NTH * k), r = e / D, c = e % D;
     *reinterpret_cast<uint2*>(dst + r * Bw<D>::LD + c) =
         make_uint2(pack_bf16(acc[k].x, acc[k].y), pack_bf16(acc[k].z, acc[k].w));
   }
@@ -489,19 +489,24 @@ struct QArgs {
   int H, N, Npad, Nb, kc, kn, phi_elu1;
 };
 
+// 8 warps: warp w takes rows 16 (w & 3) .. + 15 of the query block and keys
+// 32 (w >> 2) .. + 31 of each critical key block; the two key halves' partial
+// dQ are summed through shared memory, then the first half's warps add the
+// linear branch and store.
 template <int D>
-__global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
+__global__ void __launch_bounds__(256, 1) bwd_q_kernel(const QArgs a) {
   using T = Bw<D>;
   constexpr int NT = T::NT;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   bf16* Qs = reinterpret_cast<bf16*>(smem_raw);
   bf16* dOs = Qs + T::kTile;
   bf16* dns = dOs + T::kTile;  // dnum tile
-  bf16* KVs = dns + T::kTile;  // [2 buffers][K tile, V tile]
+  bf16* KVs = dns + T::kTile;  // [2 buffers][K tile, V tile]; after the loop: dQ partials
   bf16* Hs = KVs + 4 * T::kTile;  // [D][LD]: H_i
   float* zis = reinterpret_cast<float*>(Hs + T::kMat);  // [D]: Z_i
   const int i = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int rg = warp & 3, kh = warp >> 2;  // row group, key half
   const int t0 = i * 64, nv = min(64, a.N - t0);
   const float asc = a.alpha ? a.alpha[bh % a.H] : 1.0f;  // dO^s = asc dO
   const bool linear = a.kc + a.kn < a.Nb;
@@ -524,11 +529,11 @@ __global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
   // H_i = H_tot - sum over the excluded blocks of h_j, Z_i likewise (while the
   // first tiles land)
   if (linear)
-    complement_sum<D>(Hs, zis, a.htot + size_t(bh) * D * D, a.hblk + size_t(bh) * a.Nb * D * D,
-                      a.ztot + size_t(bh) * D, a.zblk + size_t(bh) * a.Nb * D, crit, a.kc,
-                      a.neg + (size_t(bh) * a.Nb + i) * a.kn, a.kn);
+    complement_sum<D, 256>(Hs, zis, a.htot + size_t(bh) * D * D, a.hblk + size_t(bh) * a.Nb * D * D,
+                           a.ztot + size_t(bh) * D, a.zblk + size_t(bh) * a.Nb * D, crit, a.kc,
+                           a.neg + (size_t(bh) * a.Nb + i) * a.kn, a.kn);
 
-  const int r0 = warp * 16, ra = r0 + g, rb = ra + 8;
+  const int r0 = rg * 16, ra = r0 + g, rb = ra + 8;
   const bool va = ra < nv, vb = rb < nv;
   const float lse2a = va ? a.lse[rowbase + ra] * kLog2e : INFINITY;
   const float lse2b = vb ? a.lse[rowbase + rb] * kLog2e : INFINITY;
@@ -545,31 +550,49 @@ __global__ void __launch_bounds__(128) bwd_q_kernel(const QArgs a) {
       cp_async_wait<0>();
     }
     __syncthreads();
-    const bf16* Ks = KVs + (t & 1) * 2 * T::kTile;
+    const bf16* Ks = KVs + (t & 1) * 2 * T::kTile + kh * 32 * T::LD;  // this warp's 32 keys
     const bf16* Vs = Ks + T::kTile;
-    const int nvj = min(64, a.N - crit[t] * 64);
-    float s[8][4], dp[8][4];
+    const int nvj = min(64, a.N - crit[t] * 64) - kh * 32;
+    float s[4][4], dp[4][4];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.0f;
-    mma_xyt<8, D>(s, Qs, T::LD, r0, Ks, T::LD, lane);
-    mma_xyt<8, D>(dp, dOs, T::LD, r0, Vs, T::LD, lane);
+    mma_xyt<4, D>(s, Qs, T::LD, r0, Ks, T::LD, lane);
+    mma_xyt<4, D>(dp, dOs, T::LD, r0, Vs, T::LD, lane);
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int key = nt * 8 + 2 * q + (e & 1);
         const float p = key < nvj ? ex2_approx(fmaf(s[nt][e], a.scale_log2, -(e < 2 ? lse2a : lse2b))) : 0.0f;
         s[nt][e] = p * (asc * dp[nt][e] - (e < 2 ? Da : Db));  // dS
       }
-    mma_pz<NT>(dq, s, Ks, T::LD, lane);
+    mma_pz<NT, 2>(dq, s, Ks, T::LD, lane);
     __syncthreads();  // this buffer is refilled two pairs on
   }
+  // the two key halves' partial dQ: the second half's warps hand theirs over
+  float* red = reinterpret_cast<float*>(KVs);  // [4 row groups][16 rows][D]
+  if (kh == 1) {
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt) {
+      const int c = nt * 8 + 2 * q;
+      *reinterpret_cast<float2*>(red + (r0 + g) * D + c) = make_float2(dq[nt][0], dq[nt][1]);
+      *reinterpret_cast<float2*>(red + (r0 + g + 8) * D + c) = make_float2(dq[nt][2], dq[nt][3]);
+    }
+  }
+  __syncthreads();
+  if (kh == 1) return;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) dq[nt][e] *= a.scale;
+  for (int nt = 0; nt < NT; ++nt) {
+    const int c = nt * 8 + 2 * q;
+    const float2 x0 = *reinterpret_cast<const float2*>(red + (r0 + g) * D + c);
+    const float2 x1 = *reinterpret_cast<const float2*>(red + (r0 + g + 8) * D + c);
+    dq[nt][0] = (dq[nt][0] + x0.x) * a.scale;
+    dq[nt][1] = (dq[nt][1] + x0.y) * a.scale;
+    dq[nt][2] = (dq[nt][2] + x1.x) * a.scale;
+    dq[nt][3] = (dq[nt][3] + x1.y) * a.scale;
+  }
 
   if (linear) {
     // dphi(Q_i) = dnum H_i^T + dden Z_i^T, through the feature map's Jacobian
@@ -612,21 +635,26 @@ struct KVArgs {
   int H, N, Npad, Nb, linear, phi_elu1;
 };
 
+// 8 warps: warp w takes key rows 16 (w & 3) .. + 15 of the key block and
+// queries 32 (w >> 2) .. + 31 of each query block; the two query halves'
+// partial dK and dV are summed through shared memory, then the first half's
+// warps add the linear branch and store.
 template <int D>
-__global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
+__global__ void __launch_bounds__(256, 1) bwd_kv_kernel(const KVArgs a) {
   using T = Bw<D>;
   constexpr int NT = T::NT;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   bf16* Ks = reinterpret_cast<bf16*>(smem_raw);
   bf16* Vs = Ks + T::kTile;
   bf16* PKs = Vs + T::kTile;
-  bf16* QOs = PKs + T::kTile;     // [2 buffers][Q tile, dO tile]
+  bf16* QOs = PKs + T::kTile;     // [2 buffers][Q tile, dO tile]; after the loop: dK, dV partials
   bf16* As = QOs + 4 * T::kTile;  // [D][LD]: A_j
   float* bjs = reinterpret_cast<float*>(As + T::kMat);  // [D]
   float* lse2s = bjs + D;                               // [2][64]
   float* Ds = lse2s + 128;                              // [2][64]
   const int j = blockIdx.x, bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int rg = warp & 3, qh = warp >> 2;  // key-row group, query half
   const int t0 = j * 64, nvj = min(64, a.N - t0);
   const float asc = a.alpha ? a.alpha[bh % a.H] : 1.0f;  // dO^s = asc dO
   const size_t rowbase = size_t(bh) * a.Npad + t0;
@@ -655,11 +683,11 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
   // A_j = dH_tot - sum over the query blocks that exclude j of dH_i, b_j likewise
   if (a.linear) {
     const int nE = a.cntE[size_t(bh) * a.Nb + j];
-    complement_sum<D>(As, bjs, a.dhtot + size_t(bh) * D * D, a.dhblk + size_t(bh) * a.Nb * D * D,
-                      a.dztot + size_t(bh) * D, a.dzblk + size_t(bh) * a.Nb * D,
-                      a.colE + (size_t(bh) * a.Nb + j) * a.Nb, nE, nullptr, 0);
+    complement_sum<D, 256>(As, bjs, a.dhtot + size_t(bh) * D * D, a.dhblk + size_t(bh) * a.Nb * D * D,
+                           a.dztot + size_t(bh) * D, a.dzblk + size_t(bh) * a.Nb * D,
+                           a.colE + (size_t(bh) * a.Nb + j) * a.Nb, nE, nullptr, 0);
   }
-  const int r0 = warp * 16, ra = r0 + g, rb = ra + 8;
+  const int r0 = rg * 16, ra = r0 + g, rb = ra + 8;
   const bool va = ra < nvj, vb = rb < nvj;
 
   float dk[NT][4], dv[NT][4];
@@ -675,45 +703,69 @@ __global__ void __launch_bounds__(128) bwd_kv_kernel(const KVArgs a) {
       cp_async_wait<0>();
     }
     __syncthreads();
-    const bf16* Qs = QOs + (t & 1) * 2 * T::kTile;
+    const bf16* Qs = QOs + (t & 1) * 2 * T::kTile + qh * 32 * T::LD;  // this warp's 32 queries
     const bf16* dOs = Qs + T::kTile;
-    const float* l2 = lse2s + (t & 1) * 64;
-    const float* Dc = Ds + (t & 1) * 64;
-    float st[8][4], dpt[8][4];
+    const float* l2 = lse2s + (t & 1) * 64 + qh * 32;
+    const float* Dc = Ds + (t & 1) * 64 + qh * 32;
+    float st[4][4], dpt[4][4];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) st[nt][e] = dpt[nt][e] = 0.0f;
-    mma_xyt<8, D>(st, Ks, T::LD, r0, Qs, T::LD, lane);  // S^T = K_j Q_i^T
+    mma_xyt<4, D>(st, Ks, T::LD, r0, Qs, T::LD, lane);  // S^T = K_j Q_i^T
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int col = nt * 8 + 2 * q + (e & 1);
         const bool vk = e < 2 ? va : vb;
         st[nt][e] = vk ? ex2_approx(fmaf(st[nt][e], a.scale_log2, -l2[col])) : 0.0f;  // P^T
       }
-    mma_pz<NT>(dv, st, dOs, T::LD, lane);                 // dV += P^T dO_i
-    mma_xyt<8, D>(dpt, Vs, T::LD, r0, dOs, T::LD, lane);  // dP^T = V_j dO_i^T
+    mma_pz<NT, 2>(dv, st, dOs, T::LD, lane);              // dV += P^T dO_i
+    mma_xyt<4, D>(dpt, Vs, T::LD, r0, dOs, T::LD, lane);  // dP^T = V_j dO_i^T
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int col = nt * 8 + 2 * q + (e & 1);
         st[nt][e] *= asc * dpt[nt][e] - Dc[col];  // dS^T
       }
-    mma_pz<NT>(dk, st, Qs, T::LD, lane);  // dK += dS^T Q_i
+    mma_pz<NT, 2>(dk, st, Qs, T::LD, lane);  // dK += dS^T Q_i
     __syncthreads();  // this buffer is refilled two pairs on
   }
   cp_async_wait<0>();
   __syncthreads();  // K, V, phi(K) and A_j are in place even without a sparse pair
+  // the two query halves' partials: the second half's warps hand theirs over
+  float* redk = reinterpret_cast<float*>(QOs);  // [4 row groups][16 rows][D]
+  float* redv = redk + 64 * D;
+  if (qh == 1) {
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      dv[nt][e] *= asc;
-      dk[nt][e] *= a.scale;
+    for (int nt = 0; nt < NT; ++nt) {
+      const int c = nt * 8 + 2 * q;
+      *reinterpret_cast<float2*>(redk + (r0 + g) * D + c) = make_float2(dk[nt][0], dk[nt][1]);
+      *reinterpret_cast<float2*>(redk + (r0 + g + 8) * D + c) = make_float2(dk[nt][2], dk[nt][3]);
+      *reinterpret_cast<float2*>(redv + (r0 + g) * D + c) = make_float2(dv[nt][0], dv[nt][1]);
+      *reinterpret_cast<float2*>(redv + (r0 + g + 8) * D + c) = make_float2(dv[nt][2], dv[nt][3]);
     }
+  }
+  __syncthreads();
+  if (qh == 1) return;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int c = nt * 8 + 2 * q;
+    const float2 k0 = *reinterpret_cast<const float2*>(redk + (r0 + g) * D + c);
+    const float2 k1 = *reinterpret_cast<const float2*>(redk + (r0 + g + 8) * D + c);
+    const float2 v0 = *reinterpret_cast<const float2*>(redv + (r0 + g) * D + c);
+    const float2 v1 = *reinterpret_cast<const float2*>(redv + (r0 + g + 8) * D + c);
+    dk[nt][0] = (dk[nt][0] + k0.x) * a.scale;
+    dk[nt][1] = (dk[nt][1] + k0.y) * a.scale;
+    dk[nt][2] = (dk[nt][2] + k1.x) * a.scale;
+    dk[nt][3] = (dk[nt][3] + k1.y) * a.scale;
+    dv[nt][0] = (dv[nt][0] + v0.x) * asc;
+    dv[nt][1] = (dv[nt][1] + v0.y) * asc;
+    dv[nt][2] = (dv[nt][2] + v1.x) * asc;
+    dv[nt][3] = (dv[nt][3] + v1.y) * asc;
+  }
 
   if (a.linear) {
     mma_xz<NT, D>(dv, PKs, T::LD, r0, As, T::LD, lane);  // dV += phi(K_j) A_j
@@ -803,7 +855,7 @@ cudaError_t run_backward(const BwdArgs& a, cudaStream_t s) {
     const int bytes = (7 * T::kTile + T::kMat) * 2 + D * 4;
     e = set_smem(bwd_q_kernel<D>, bytes);
     if (e == cudaSuccess) {
-      bwd_q_kernel<D><<<blocks, 128, bytes, s>>>(qa);
+      bwd_q_kernel<D><<<blocks, 256, bytes, s>>>(qa);
       e = cudaGetLastError();
     }
   }
@@ -815,7 +867,7 @@ cudaError_t run_backward(const BwdArgs& a, cudaStream_t s) {
     const int bytes = (7 * T::kTile + T::kMat) * 2 + (D + 256) * 4;
     e = set_smem(bwd_kv_kernel<D>, bytes);
     if (e == cudaSuccess) {
-      bwd_kv_kernel<D><<<blocks, 128, bytes, s>>>(ka);
+      bwd_kv_kernel<D><<<blocks, 256, bytes, s>>>(ka);
       e = cudaGetLastError();
     }
   }
