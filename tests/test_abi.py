@@ -139,3 +139,51 @@ def test_binding_fails_loudly_without_library(tmp_path):
             mod.load(str(tmp_path / "missing.so"))
         finally:
             mod._lib = saved
+
+
+def test_router_training_and_backward_reject_on_host(lib):
+    # Fake device addresses again: every case below is rejected before any CUDA call.
+    by = ctypes.byref
+    p = params()
+    nb = sla.workspace_size(p)
+    # SoftTop-k router
+    assert lib.sla_router_soft_topk(0x10000, 0x20000, by(p), 0.0, 0x60000, None, None, 0x50000, nb, None) == \
+        sla.SLA_ERR_INVALID_ARG
+    assert lib.sla_router_soft_topk(0x10000, 0x20000, by(p), float("inf"), 0x60000, None, None, 0x50000, nb,
+                                    None) == sla.SLA_ERR_INVALID_ARG
+    assert lib.sla_router_soft_topk(0x10000, 0x20000, by(p), 0.1, None, None, None, 0x50000, nb, None) == \
+        sla.SLA_ERR_INVALID_ARG
+    assert lib.sla_router_soft_topk(0x10008, 0x20000, by(p), 0.1, 0x60000, None, None, 0x50000, nb, None) == \
+        sla.SLA_ERR_ALIGNMENT
+    assert lib.sla_router_soft_topk(0x10000, 0x20000, by(p), 0.1, 0x60000, None, None, 0x50000, nb - 1, None) == \
+        sla.SLA_ERR_WORKSPACE
+    # training forward
+    sv = sla.Saved(o_s=0x70000, o_l=0x80000, lse=0x90000, den=0xA0000)
+    tf = lambda pp, s_, n=nb: lib.sla_forward_train(0x10000, 0x20000, 0x30000, 0x40000, by(pp), s_, 0x50000,  # noqa: E731
+                                                    n, None)
+    assert tf(p, None) == sla.SLA_ERR_INVALID_ARG
+    assert tf(p, by(sla.Saved(o_s=0x70000, o_l=None, lse=0x90000, den=0xA0000))) == sla.SLA_ERR_INVALID_ARG
+    assert tf(p, by(sla.Saved(o_s=0x70008, o_l=0x80000, lse=0x90000, den=0xA0000))) == sla.SLA_ERR_ALIGNMENT
+    assert tf(p, by(sv), nb - 1) == sla.SLA_ERR_WORKSPACE
+    pq = params(precision="i8qk_f8pv", variant="sla2", k_neg=0)
+    pq.alpha = 0x1000
+    assert tf(pq, by(sv), 1 << 30) == sla.SLA_ERR_UNSUPPORTED
+    # backward
+    bn = lib.sla_backward_workspace_size(by(p))
+    assert bn > 0 and lib.sla_backward_workspace_size(by(params(k_crit=0))) == 0
+
+    def bw(pp, dO=0xB0000, saved=sv, fb=nb, dW=None, da=None, bnb=bn):
+        return lib.sla_backward(0x10000, 0x20000, 0x30000, dO, by(pp), by(saved) if saved is not None else None,
+                                0x50000, fb, 0xC0000, 0xD0000, 0xE0000, dW, da, 0xF0000, bnb, None)
+
+    assert bw(p, dO=None) == sla.SLA_ERR_INVALID_ARG
+    assert bw(p, saved=None) == sla.SLA_ERR_INVALID_ARG
+    assert bw(p, da=0x100000) == sla.SLA_ERR_INVALID_ARG  # dalpha is SLA2's
+    assert bw(p, fb=nb - 1) == sla.SLA_ERR_WORKSPACE
+    assert bw(p, bnb=bn - 1) == sla.SLA_ERR_WORKSPACE
+    assert bw(p, dO=0xB0008) == sla.SLA_ERR_ALIGNMENT
+    p2 = params(variant="sla2", k_neg=0)
+    p2.alpha = 0x1000
+    bn2 = lib.sla_backward_workspace_size(by(p2))
+    assert bw(p2, dW=0x100000, bnb=bn2, fb=sla.workspace_size(p2)) == sla.SLA_ERR_INVALID_ARG  # dW is SLA's
+    assert bw(pq, fb=1 << 30, bnb=1 << 30) == sla.SLA_ERR_UNSUPPORTED
