@@ -43,7 +43,7 @@ LOWBIT_OVER_BF16 = 2.0
 # DRAM bytes (read + write) of one attention launch, from the ncu capture
 # summarised in profiles/attn_tc_kernel_sla_wan13b_b1h12n32768d128.md; keyed by
 # workload and valid only for the attention kernel that capture was taken of
-ATTN_TRAFFIC = {"sla_wan13b_b1h12n32768d128_s95": 425895936 + 91530496}
+ATTN_TRAFFIC = {"sla_wan13b_b1h12n32768d128_s95": 421516288 + 91559424}
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "ms/forward and dense-equiv TFLOPS at 95-97% sparsity; tensor-pipe % of B200 peak"
 UNIT = "TFLOPS (dense-equivalent)"

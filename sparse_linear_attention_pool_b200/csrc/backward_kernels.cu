@@ -572,13 +572,15 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(const QArgs a) {
     __syncthreads();  // this buffer is refilled two pairs on
   }
   // the two key halves' partial dQ: the second half's warps hand theirs over
-  float* red = reinterpret_cast<float*>(KVs);  // [4 row groups][16 rows][D]
+  // (rows D + 4 floats apart, so a fragment's eight rows fall in distinct banks)
+  constexpr int RS = D + 4;
+  float* red = reinterpret_cast<float*>(KVs);  // [64 rows][RS]
   if (kh == 1) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int c = nt * 8 + 2 * q;
-      *reinterpret_cast<float2*>(red + (r0 + g) * D + c) = make_float2(dq[nt][0], dq[nt][1]);
-      *reinterpret_cast<float2*>(red + (r0 + g + 8) * D + c) = make_float2(dq[nt][2], dq[nt][3]);
+      *reinterpret_cast<float2*>(red + (r0 + g) * RS + c) = make_float2(dq[nt][0], dq[nt][1]);
+      *reinterpret_cast<float2*>(red + (r0 + g + 8) * RS + c) = make_float2(dq[nt][2], dq[nt][3]);
     }
   }
   __syncthreads();
@@ -586,8 +588,8 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(const QArgs a) {
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int c = nt * 8 + 2 * q;
-    const float2 x0 = *reinterpret_cast<const float2*>(red + (r0 + g) * D + c);
-    const float2 x1 = *reinterpret_cast<const float2*>(red + (r0 + g + 8) * D + c);
+    const float2 x0 = *reinterpret_cast<const float2*>(red + (r0 + g) * RS + c);
+    const float2 x1 = *reinterpret_cast<const float2*>(red + (r0 + g + 8) * RS + c);
     dq[nt][0] = (dq[nt][0] + x0.x) * a.scale;
     dq[nt][1] = (dq[nt][1] + x0.y) * a.scale;
     dq[nt][2] = (dq[nt][2] + x1.x) * a.scale;
@@ -736,16 +738,18 @@ __global__ void __launch_bounds__(256, 1) bwd_kv_kernel(const KVArgs a) {
   cp_async_wait<0>();
   __syncthreads();  // K, V, phi(K) and A_j are in place even without a sparse pair
   // the two query halves' partials: the second half's warps hand theirs over
-  float* redk = reinterpret_cast<float*>(QOs);  // [4 row groups][16 rows][D]
-  float* redv = redk + 64 * D;
+  // (rows D + 4 floats apart, so a fragment's eight rows fall in distinct banks)
+  constexpr int RS = D + 4;
+  float* redk = reinterpret_cast<float*>(QOs);  // [64 rows][RS]
+  float* redv = redk + 64 * RS;
   if (qh == 1) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int c = nt * 8 + 2 * q;
-      *reinterpret_cast<float2*>(redk + (r0 + g) * D + c) = make_float2(dk[nt][0], dk[nt][1]);
-      *reinterpret_cast<float2*>(redk + (r0 + g + 8) * D + c) = make_float2(dk[nt][2], dk[nt][3]);
-      *reinterpret_cast<float2*>(redv + (r0 + g) * D + c) = make_float2(dv[nt][0], dv[nt][1]);
-      *reinterpret_cast<float2*>(redv + (r0 + g + 8) * D + c) = make_float2(dv[nt][2], dv[nt][3]);
+      *reinterpret_cast<float2*>(redk + (r0 + g) * RS + c) = make_float2(dk[nt][0], dk[nt][1]);
+      *reinterpret_cast<float2*>(redk + (r0 + g + 8) * RS + c) = make_float2(dk[nt][2], dk[nt][3]);
+      *reinterpret_cast<float2*>(redv + (r0 + g) * RS + c) = make_float2(dv[nt][0], dv[nt][1]);
+      *reinterpret_cast<float2*>(redv + (r0 + g + 8) * RS + c) = make_float2(dv[nt][2], dv[nt][3]);
     }
   }
   __syncthreads();
@@ -753,10 +757,10 @@ __global__ void __launch_bounds__(256, 1) bwd_kv_kernel(const KVArgs a) {
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int c = nt * 8 + 2 * q;
-    const float2 k0 = *reinterpret_cast<const float2*>(redk + (r0 + g) * D + c);
-    const float2 k1 = *reinterpret_cast<const float2*>(redk + (r0 + g + 8) * D + c);
-    const float2 v0 = *reinterpret_cast<const float2*>(redv + (r0 + g) * D + c);
-    const float2 v1 = *reinterpret_cast<const float2*>(redv + (r0 + g + 8) * D + c);
+    const float2 k0 = *reinterpret_cast<const float2*>(redk + (r0 + g) * RS + c);
+    const float2 k1 = *reinterpret_cast<const float2*>(redk + (r0 + g + 8) * RS + c);
+    const float2 v0 = *reinterpret_cast<const float2*>(redv + (r0 + g) * RS + c);
+    const float2 v1 = *reinterpret_cast<const float2*>(redv + (r0 + g + 8) * RS + c);
     dk[nt][0] = (dk[nt][0] + k0.x) * a.scale;
     dk[nt][1] = (dk[nt][1] + k0.y) * a.scale;
     dk[nt][2] = (dk[nt][2] + k1.x) * a.scale;
