@@ -16,10 +16,11 @@
 //            then the feature map's Jacobian.
 // H_i and A_j are formed by complement, as in the forward: H_i = H_tot -
 // sum over the excluded blocks of h_j, A_j = dH_tot - sum over the query
-// blocks that exclude j of dH_i, with h_j and dH_i kept per block (d x d
-// fp32). Every product runs on the tensor cores (mma.sync m16n8k16, bf16 in,
-// fp32 accumulate); every reduction runs in a fixed order, so the gradients
-// are bitwise reproducible.
+// blocks that exclude j of dH_i, with h_j and dH_i kept per block (d x d,
+// stored in bf16 and summed in fp32: H_i and A_j enter the tensor cores in
+// bf16 anyway). Every product runs on the tensor cores (mma.sync m16n8k16,
+// bf16 in, fp32 accumulate); every reduction runs in a fixed order, so the
+// gradients are bitwise reproducible.
 #include "sla_internal.cuh"
 
 namespace sla {
@@ -234,9 +235,10 @@ __device__ __forceinline__ void store_frag_rows(bf16* dst, int D, int ra, bool v
 // ---------------------------------------------------------------------------
 // per-block X^T Y: out[bh][blk] = sum over the block's valid rows of x_r^T y_r
 // ---------------------------------------------------------------------------
-template <int D>
+// out is float32, or bf16 for the matrices only the complement sums read
+template <int D, typename OutT>
 __global__ void __launch_bounds__(2 * D) block_xty_kernel(const bf16* __restrict__ X, const bf16* __restrict__ Y,
-                                                          float* __restrict__ out, int N, int Npad, int Nb) {
+                                                          OutT* __restrict__ out, int N, int Npad, int Nb) {
   using T = Bw<D>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   bf16* Xs = reinterpret_cast<bf16*>(smem_raw);
@@ -265,23 +267,31 @@ __global__ void __launch_bounds__(2 * D) block_xty_kernel(const bf16* __restrict
     for (int nt = 0; nt < T::NT; ++nt)
       mma16816(acc[nt], a, pair_col(Ys, T::LD, k0 + 2 * q, nt * 8 + g), pair_col(Ys, T::LD, k0 + 8 + 2 * q, nt * 8 + g));
   }
-  float* o = out + (size_t(bh) * Nb + blk) * D * D;
+  OutT* o = out + (size_t(bh) * Nb + blk) * D * D;
 #pragma unroll
   for (int nt = 0; nt < T::NT; ++nt) {
     const int c = nt * 8 + 2 * q;
-    *reinterpret_cast<float2*>(o + (m0 + g) * D + c) = make_float2(acc[nt][0], acc[nt][1]);
-    *reinterpret_cast<float2*>(o + (m0 + g + 8) * D + c) = make_float2(acc[nt][2], acc[nt][3]);
+    if constexpr (sizeof(OutT) == 4) {
+      *reinterpret_cast<float2*>(o + (m0 + g) * D + c) = make_float2(acc[nt][0], acc[nt][1]);
+      *reinterpret_cast<float2*>(o + (m0 + g + 8) * D + c) = make_float2(acc[nt][2], acc[nt][3]);
+    } else {
+      *reinterpret_cast<uint32_t*>(o + (m0 + g) * D + c) = pack_bf16(acc[nt][0], acc[nt][1]);
+      *reinterpret_cast<uint32_t*>(o + (m0 + g + 8) * D + c) = pack_bf16(acc[nt][2], acc[nt][3]);
+    }
   }
 }
 
-// out[o][e] = sum over b (ascending) of in[o][b][e]
-__global__ void __launch_bounds__(256) reduce_blocks_kernel(const float* __restrict__ in, float* __restrict__ out,
+// out[o][e] = sum over b (ascending) of in[o][b][e], in float32
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(bf16 x) { return __bfloat162float(x); }
+template <typename InT>
+__global__ void __launch_bounds__(256) reduce_blocks_kernel(const InT* __restrict__ in, float* __restrict__ out,
                                                             int nb, int E) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x, o = blockIdx.y;
   if (e >= E) return;
-  const float* p = in + size_t(o) * nb * E + e;
+  const InT* p = in + size_t(o) * nb * E + e;
   float s = 0.0f;
-  for (int b = 0; b < nb; ++b) s += p[size_t(b) * E];
+  for (int b = 0; b < nb; ++b) s += to_f32(p[size_t(b) * E]);
   out[size_t(o) * E + e] = s;
 }
 
@@ -437,13 +447,13 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(const PrepArgs a) {
   }
 }
 
-// dst (bf16 [D][LD] tile) = tot - sum over the listed blocks of blk[j] (fp32
-// d x d each), and zdst[c] = ztot[c] - sum of zblk[j][c]: the complement sums
+// dst (bf16 [D][LD] tile) = tot - sum over the listed blocks of blk[j] (bf16
+// d x d each, summed in fp32), and zdst[c] = ztot[c] - sum of zblk[j][c]: the complement sums
 // of H_i, Z_i (query side) and A_j, b_j (key side). Each of the NTH threads
 // keeps its D * D / NTH entries in registers and subtracts block after block (coalesced
 // float4 loads, independent across the thread's entries), in list order.
 template <int D, int NTH>
-__device__ __forceinline__ void complement_sum(bf16* dst, float* zdst, const float* tot, const float* blk,
+__device__ __forceinline__ void complement_sum(bf16* dst, float* zdst, const float* tot, const bf16* blk,
                                                const float* ztot, const float* zblk, const int32_t* l1, int n1,
                                                const int32_t* l2, int n2) {
   constexpr int PER = D * D / 4 / NTH;
@@ -454,14 +464,14 @@ __device__ __forceinline__ void complement_sum(bf16* dst, float* zdst, const flo
   for (int k = 0; k < PER; ++k) acc[k] = t4[tid + NTH * k];
   float z = tid < D ? ztot[tid] : 0.0f;
   auto sub = [&](int j) {
-    const float4* b4 = reinterpret_cast<const float4*>(blk + size_t(j) * D * D);
+    const uint2* b4 = reinterpret_cast<const uint2*>(blk + size_t(j) * D * D);  // 4 bf16 per load
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
-      const float4 v = b4[tid + NTH * k];
-      acc[k].x -= v.x;
-      acc[k].y -= v.y;
-      acc[k].z -= v.z;
-      acc[k].w -= v.w;
+      const uint2 v = b4[tid + NTH * k];
+      acc[k].x -= bf16_lo(v.x);
+      acc[k].y -= bf16_hi(v.x);
+      acc[k].z -= bf16_lo(v.y);
+      acc[k].w -= bf16_hi(v.y);
     }
     if (tid < D) z -= zblk[size_t(j) * D + tid];
   };
@@ -482,7 +492,9 @@ __device__ __forceinline__ void complement_sum(bf16* dst, float* zdst, const flo
 struct QArgs {
   const bf16 *Q, *K, *V, *dO, *dnum;
   const int32_t *crit, *neg;
-  const float *lse, *Drow, *dden, *htot, *hblk, *ztot, *zblk;
+  const float *lse, *Drow, *dden, *htot;
+  const bf16* hblk;
+  const float *ztot, *zblk;
   const float* alpha;  // SLA2 [H] (dO^s = alpha dO); null for SLA
   bf16* dQ;
   float scale, scale_log2;
@@ -630,7 +642,9 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(const QArgs a) {
 struct KVArgs {
   const bf16 *Q, *K, *V, *dO, *phik;
   const int *colC, *colE, *cntC, *cntE;
-  const float *lse, *Drow, *dhtot, *dhblk, *dztot, *dzblk;
+  const float *lse, *Drow, *dhtot;
+  const bf16* dhblk;
+  const float *dztot, *dzblk;
   const float* alpha;  // SLA2 [H]; null for SLA
   bf16 *dK, *dV;
   float scale, scale_log2;
@@ -714,7 +728,8 @@ __global__ void __launch_bounds__(256, 1) bwd_kv_kernel(const KVArgs a) {
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) st[nt][e] = dpt[nt][e] = 0.0f;
-    mma_xyt<4, D>(st, Ks, T::LD, r0, Qs, T::LD, lane);  // S^T = K_j Q_i^T
+    mma_xyt<4, D>(st, Ks, T::LD, r0, Qs, T::LD, lane);    // S^T = K_j Q_i^T
+    mma_xyt<4, D>(dpt, Vs, T::LD, r0, dOs, T::LD, lane);  // dP^T = V_j dO_i^T
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -723,8 +738,7 @@ __global__ void __launch_bounds__(256, 1) bwd_kv_kernel(const KVArgs a) {
         const bool vk = e < 2 ? va : vb;
         st[nt][e] = vk ? ex2_approx(fmaf(st[nt][e], a.scale_log2, -l2[col])) : 0.0f;  // P^T
       }
-    mma_pz<NT, 2>(dv, st, dOs, T::LD, lane);              // dV += P^T dO_i
-    mma_xyt<4, D>(dpt, Vs, T::LD, r0, dOs, T::LD, lane);  // dP^T = V_j dO_i^T
+    mma_pz<NT, 2>(dv, st, dOs, T::LD, lane);  // dV += P^T dO_i
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -831,23 +845,24 @@ cudaError_t run_backward(const BwdArgs& a, cudaStream_t s) {
     e = cudaGetLastError();
   }
   const int xty_bytes = 2 * T::kTile * 2;
-  if (e == cudaSuccess) e = set_smem(block_xty_kernel<D>, xty_bytes);
+  if (e == cudaSuccess) e = set_smem(block_xty_kernel<D, bf16>, xty_bytes);
+  if (e == cudaSuccess) e = set_smem(block_xty_kernel<D, float>, xty_bytes);
   if (e == cudaSuccess && L.linear) {
     // 3. h_j = phi(K_j)^T V_j and dH_i = phi(Q_i)^T dnum_i per block, their head totals
-    block_xty_kernel<D><<<blocks, 2 * D, xty_bytes, s>>>(a.phik, a.V, a.hblk, L.N, L.Npad, Nb);
-    block_xty_kernel<D><<<blocks, 2 * D, xty_bytes, s>>>(a.phiq, a.dnum, a.dhblk, L.N, L.Npad, Nb);
-    reduce_blocks_kernel<<<dim3((D * D + 255) / 256, BH), 256, 0, s>>>(a.dhblk, a.dhtot, Nb, D * D);
-    reduce_blocks_kernel<<<dim3((D + 255) / 256, BH), 256, 0, s>>>(a.dzblk, a.dztot, Nb, D);
+    block_xty_kernel<D, bf16><<<blocks, 2 * D, xty_bytes, s>>>(a.phik, a.V, a.hblk, L.N, L.Npad, Nb);
+    block_xty_kernel<D, bf16><<<blocks, 2 * D, xty_bytes, s>>>(a.phiq, a.dnum, a.dhblk, L.N, L.Npad, Nb);
+    reduce_blocks_kernel<bf16><<<dim3((D * D + 255) / 256, BH), 256, 0, s>>>(a.dhblk, a.dhtot, Nb, D * D);
+    reduce_blocks_kernel<float><<<dim3((D + 255) / 256, BH), 256, 0, s>>>(a.dzblk, a.dztot, Nb, D);
     e = cudaGetLastError();
   }
   // 4. dW = sum over rows of O^l^T dO (SLA), dalpha_h = sum of the partials (SLA2)
   if (e == cudaSuccess && a.dW != nullptr) {
-    block_xty_kernel<D><<<blocks, 2 * D, xty_bytes, s>>>(a.save_ol, a.dO, a.dwpart, L.N, L.Npad, Nb);
-    reduce_blocks_kernel<<<dim3((D * D + 255) / 256, 1), 256, 0, s>>>(a.dwpart, a.dW, BH * Nb, D * D);
+    block_xty_kernel<D, float><<<blocks, 2 * D, xty_bytes, s>>>(a.save_ol, a.dO, a.dwpart, L.N, L.Npad, Nb);
+    reduce_blocks_kernel<float><<<dim3((D * D + 255) / 256, 1), 256, 0, s>>>(a.dwpart, a.dW, BH * Nb, D * D);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess && a.dalpha != nullptr) {
-    reduce_blocks_kernel<<<dim3(1, L.H), 256, 0, s>>>(a.dapart, a.dalpha, L.B * Nb, 1);
+    reduce_blocks_kernel<float><<<dim3(1, L.H), 256, 0, s>>>(a.dapart, a.dalpha, L.B * Nb, 1);
     e = cudaGetLastError();
   }
   const float scale = a.scale;

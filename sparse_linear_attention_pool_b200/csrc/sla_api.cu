@@ -256,8 +256,8 @@ sla_status sla_backward(const void* Q, const void* K, const void* V, const void*
   a.dden = reinterpret_cast<float*>(ws + BL.dden);
   a.dzblk = reinterpret_cast<float*>(ws + BL.dzblk);
   a.dztot = reinterpret_cast<float*>(ws + BL.dztot);
-  a.hblk = reinterpret_cast<float*>(ws + BL.hblk);
-  a.dhblk = reinterpret_cast<float*>(ws + BL.dhblk);
+  a.hblk = reinterpret_cast<__nv_bfloat16*>(ws + BL.hblk);
+  a.dhblk = reinterpret_cast<__nv_bfloat16*>(ws + BL.dhblk);
   a.dhtot = reinterpret_cast<float*>(ws + BL.dhtot);
   a.dwpart = reinterpret_cast<float*>(ws + BL.dwpart);
   a.dapart = reinterpret_cast<float*>(ws + BL.dapart);

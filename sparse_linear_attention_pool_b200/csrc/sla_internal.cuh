@@ -175,8 +175,8 @@ inline BwLayout make_bw_layout(const sla_params& p) {
   L.dden = take(rows * 4);                   // -(dO^l . O^l) / den
   L.dzblk = take(BH * Nb * d * 4);           // dZ_i
   L.dztot = take(BH * d * 4);
-  L.hblk = take(L.linear ? BH * Nb * d * d * 4 : 0);   // h_j
-  L.dhblk = take(L.linear ? BH * Nb * d * d * 4 : 0);  // dH_i
+  L.hblk = take(L.linear ? BH * Nb * d * d * 2 : 0);   // h_j, bf16
+  L.dhblk = take(L.linear ? BH * Nb * d * d * 2 : 0);  // dH_i, bf16
   L.dhtot = take(BH * d * d * 4);
   L.dwpart = take(L.sla ? BH * Nb * d * d * 4 : 0);    // per-block O^l^T dO
   L.dapart = take(BH * Nb * 4);                        // per-block dO . (O^s - O^l), [H][B][Nb]
@@ -195,7 +195,8 @@ struct BwdArgs {
   const int8_t* mc;
   const int32_t *crit, *neg;
   __nv_bfloat16 *dnum, *phiq;
-  float *Drow, *dden, *dzblk, *dztot, *hblk, *dhblk, *dhtot, *dwpart, *dapart;
+  float *Drow, *dden, *dzblk, *dztot, *dhtot, *dwpart, *dapart;
+  __nv_bfloat16 *hblk, *dhblk;  // per-block d x d, read only by the complement sums
   int *colC, *colE, *cntC, *cntE;
   __nv_bfloat16 *dQ, *dK, *dV;
   float *dW, *dalpha;
