@@ -1,5 +1,5 @@
 /*
- * sla.h -- C ABI of the B200 (sm_100a) SLA / SLA2 sparse-linear attention forward pass.
+ * sla.h -- C ABI of the B200 (sm_100a) SLA / SLA2 sparse-linear attention.
  *
  * One call, sla_forward(), runs the whole forward of a batch of heads on one
  * GPU, every step in this library's CUDA kernels:
@@ -16,6 +16,11 @@
  *      (online softmax, tensor cores), the linear branch
  *      phi(Q_i) H_i / phi(Q_i) Z_i over the marginal blocks, and the combine
  *      (SLA: O = O^s + O^l W; SLA2: O = alpha_h O^s + (1 - alpha_h) O^l).
+ *
+ * Beside it: sla_dense_forward() (the dense baseline), sla_router_soft_topk()
+ * (SLA2's differentiable router for its first training stage),
+ * sla_forward_train() and sla_backward() (the gradients of the forward), and
+ * read-back and timing helpers.
  *
  * Sources (page title, section):
  *   - "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable

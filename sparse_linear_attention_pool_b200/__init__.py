@@ -8,6 +8,14 @@ fallback: if the compiled library is missing, load() raises.
     o = sla.forward(q, k, v, N=N, variant="sla2", k_crit=15, alpha=alpha,
                     proj_q=wq, proj_k=wk)
 
+    # training: the forward that keeps its activations, then the gradients
+    p = sla.make_params(B, H, N, d, variant="sla2", k_crit=15, alpha=alpha, proj_q=wq, proj_k=wk)
+    o, saved, ws = sla.forward_train(q, k, v, params=p)
+    dq, dk, dv, dalpha, _ = sla.backward(q, k, v, do, params=p, saved=saved, fwd_workspace=ws)
+
+    # SLA2's SoftTop-k router (first training stage)
+    m, lam, pc, _ = sla.router_soft_topk(q, k, tau=0.01, params=p, want_pc=True)
+
 q, k, v: [B, H, N_pad, d] torch.bfloat16 CUDA tensors, N_pad = 64 * ceil(N / 64).
 """
 from __future__ import annotations
