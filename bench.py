@@ -72,8 +72,9 @@ def attention_flops(w):
     every critical 64x64 pair, phi(Q) H for the linear branch, and (SLA) O^l W."""
     BH = w.B * w.H
     sparse = BH * w.Nb * w.k_crit * 4.0 * 64 * 64 * w.d
-    linear = BH * 2.0 * w.N * w.d * w.d
-    proj = BH * 2.0 * w.N * w.d * w.d if w.variant == "sla" else 0.0
+    has_linear = w.k_crit + w.k_neg < w.Nb  # without a marginal block the kernel skips both
+    linear = BH * 2.0 * w.N * w.d * w.d if has_linear else 0.0
+    proj = BH * 2.0 * w.N * w.d * w.d if (w.variant == "sla" and has_linear) else 0.0
     return sparse + linear + proj
 
 
