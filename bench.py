@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -36,7 +37,7 @@ import numpy as np  # noqa: E402
 import workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "sla_wan13b_b1h12n32768d128_s95"
-NORTH_STAR_97 = "sla2_b1h12n32768d128_s97"
+SLA2_97_WORKLOAD = "sla2_b1h12n32768d128_s97"
 QUANT_WORKLOAD = "sla2_q_wan14b_b1h40n75600d128_s97"
 # dense tensor throughput of the 8-bit kinds relative to bf16 (2.25 vs 4.5 PFLOP/s nominal)
 LOWBIT_OVER_BF16 = 2.0
@@ -184,7 +185,9 @@ class ClockSampler:
     def __init__(self, device_index):
         self.idx = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        # the sampled clock log (CSV) goes to $SLA_BENCH_LOG_DIR, else the temp directory
+        log_dir = os.environ.get("SLA_BENCH_LOG_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(log_dir, f"sla_bench_clocks_rank{device_index}.csv")
 
     def start(self):
         try:
@@ -545,8 +548,8 @@ def run_ours(args):
         res["dense_baseline"] = {"ms": round(dense_ms, 4),
                                  "tflops": round(dense_eq_flops(w) / (dense_ms * 1e-3) / 1e12, 2),
                                  "speedup_of_sparse": round(dense_ms / ms, 3)}
-    if not args.no_north_star and rank == 0 and args.workload != NORTH_STAR_97:
-        w97 = W.WORKLOADS[NORTH_STAR_97]
+    if not args.no_sla2_97 and rank == 0 and args.workload != SLA2_97_WORKLOAD:
+        w97 = W.WORKLOADS[SLA2_97_WORKLOAD]
         inp97 = W.make_inputs(w97)
         dev97 = device_inputs(inp97)
         ms97, st97, _ = time_forward(sla, w97, dev97, args.steps, args.warmup, 1, stage_timing=True)
@@ -564,7 +567,7 @@ def run_ours(args):
                              "tflops": round(backward_flops(w97) / (b97 * 1e-3) / 1e12, 2),
                              "dense_flash_backward_ms": None if d97 is None else round(d97, 4),
                              "speedup_vs_dense_backward": None if d97 is None else round(d97 / b97, 3)}
-        res["north_star_97"] = entry
+        res["sla2_97"] = entry
         del dev97
     if not args.no_quant and rank == 0 and args.workload != QUANT_WORKLOAD:
         wq = W.WORKLOADS[QUANT_WORKLOAD]
@@ -722,7 +725,8 @@ def main():
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-only", action="store_true",
                     help="time sla_backward alone on --workload (one JSON line)")
-    ap.add_argument("--no-north-star", action="store_true")
+    ap.add_argument("--no-sla2-97", action="store_true",
+                    help="skip the SLA2 97 %% entry (forward, router, backward)")
     ap.add_argument("--no-quant", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="run the N / sparsity sweep instead of the benchmark line")
