@@ -10,8 +10,9 @@ operands: a relative error of about 2^-9 per operand, averaging down over
 the sums: measured rel-L2 4e-3 to 7.4e-3 and max-abs 5e-3 to 7.7e-3 of the
 tensor's largest entry over the cases below, the 32k-token workloads
 included. The tolerances (rel-L2 GRAD_REL_L2, max-abs against the tensor's
-own largest entry GRAD_MAX_REL) sit at about twice that; dW and dalpha are
-float32 sums of bf16 products and must match to DW_REL.
+own largest entry GRAD_MAX_REL) sit at about twice that. dW and dalpha are
+checked as exact reductions of the saved activations, and against the oracle
+(check_param_grad).
 
 The saved activations are checked too: O^s and O^l within the bf16 output
 contract, lse within LSE_ABS (fp32 log2 arithmetic), den within DEN_REL (phi
@@ -29,6 +30,8 @@ pytestmark = pytest.mark.gpu
 GRAD_REL_L2 = 1.5e-2
 GRAD_MAX_REL = 1.5e-2
 DW_REL = 1e-2
+PARAM_REL = 5e-2   # dalpha against the oracle (a cancelling sum; see check_param_grad)
+REDUCE_REL = 1e-5  # the library's float32 reductions against float64 on the same saved values
 LSE_ABS = 2e-3
 DEN_REL = 1e-2
 
@@ -105,6 +108,8 @@ CASES = [
     ("bw_all_critical", 1, 2, 64 * 5 + 7, 128, "sla", 6, 0, "softmax", True),
     ("bw_sla_no_w", 1, 1, 64 * 8 + 40, 128, "sla", 2, 1, "softmax", False),
     ("bw_one_partial_block", 1, 2, 37, 64, "sla2", 1, 0, "softmax", True),
+    ("bw_sla2_batch2_heads3", 2, 3, 64 * 7 + 21, 128, "sla2", 2, 0, "softmax", True),
+    ("bw_sla2_with_negligible", 1, 2, 64 * 10, 128, "sla2", 2, 3, "softmax", True),
 ]
 
 
@@ -117,16 +122,38 @@ def test_backward_small(cuda_lib, case, record_property):
     res = run_train(cuda_lib, inp, dO_bits, use_w)
     assert cuda_lib.read_device_status(res["fws"]) == 0
     per_head = [check_head(res, inp, idx, dO_bits, use_w, record_property) for idx in range(B * H)]
-    if variant == "sla":
+    check_param_grad(res, inp, dO_bits, per_head)
+
+
+def check_param_grad(res, inp, dO_bits, per_head):
+    """dW (SLA) and dalpha (SLA2) are sums over every row of products of the
+    saved bf16 activations with dO. They are checked as the exact reductions
+    of what the training forward saved (float64 here against the library's
+    float32 sums: REDUCE_REL of the sum of the terms' magnitudes), the saved
+    activations themselves having been checked against the oracle. dalpha
+    cancels (random-sign dO), so the activations' bf16-level errors reach it
+    at about 1 % relative; it is held to PARAM_REL against the oracle. dW does
+    not cancel that way and stays within DW_REL."""
+    w = inp.w
+    N = w.N
+    got = res["pg"].cpu().numpy().astype(np.float64)
+    Os = from_dev_bf16(res["saved"]["o_s"])[:, :, :N]
+    Ol = from_dev_bf16(res["saved"]["o_l"])[:, :, :N]
+    dO = W.bf16_bits_to_f32(dO_bits[:, :, :N]).astype(np.float64)
+    if w.variant == "sla":
+        exact = np.einsum("bhnc,bhne->ce", Ol, dO)
+        scale = np.einsum("bhnc,bhne->ce", np.abs(Ol), np.abs(dO))
+        assert np.all(np.abs(got - exact) <= REDUCE_REL * scale + 1e-6), "dW is not the reduction of O^l^T dO"
         dW = sum(r["dW"] for r in per_head)
-        got = res["pg"].cpu().numpy().astype(np.float64)
         assert rel_l2(got, dW) <= DW_REL, f"dW rel-L2 {rel_l2(got, dW):.3e}"
     else:
-        got = res["pg"].cpu().numpy().astype(np.float64)
-        for idx, r in enumerate(per_head):
-            _, h = inp.heads[idx]
+        terms = dO * (Os - Ol)
+        exact = terms.sum(axis=(0, 2, 3))
+        scale = np.abs(terms).sum(axis=(0, 2, 3))
+        assert np.all(np.abs(got - exact) <= REDUCE_REL * scale + 1e-6), (got, exact)
+        for h in range(w.H):
             want = sum(pr["dalpha"] for j, pr in enumerate(per_head) if inp.heads[j][1] == h)
-            assert got[h] == pytest.approx(want, rel=DW_REL, abs=1e-3), f"dalpha head {h}"
+            assert got[h] == pytest.approx(want, rel=PARAM_REL, abs=1e-3), f"dalpha head {h}"
 
 
 def test_training_forward_output_and_determinism(cuda_lib):

@@ -86,6 +86,7 @@ CASES = [
     ("many_tiles_hot", 1, 3, 64 * 300 + 5, 128, "sla2", 9, 0.5),
     ("nb1500_vpl64", 1, 1, 64 * 1500, 64, "sla", 45, 1e-3),
     ("nb2100_vpl128", 1, 1, 64 * 2100 - 20, 64, "sla", 63, 1e-3),
+    ("sla2_batch2_heads3", 2, 3, 64 * 9 + 5, 128, "sla2", 3, 0.02),
 ]
 
 
