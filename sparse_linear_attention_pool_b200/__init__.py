@@ -348,3 +348,38 @@ def backward(q, k, v, do, *, params: Params, saved: dict, fwd_workspace, want_pa
                              _ptr(dalpha), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "sla_backward")
     return dq, dk, dv, (dalpha if sla2 else dW), workspace
+
+
+def attention(q, k, v, *, N: Optional[int] = None, variant: str = "sla", k_crit: int, k_neg: int = 0,
+              softmax_scale: float = 0.0, w_proj=None, proj_q=None, proj_k=None, alpha=None,
+              phi: str = "softmax"):
+    """Differentiable SLA / SLA2 attention for PyTorch: the forward through
+    sla_forward_train and, on .backward(), the gradients through sla_backward
+    (mask held fixed) for q, k, v and, when they require grad, SLA's w_proj
+    and SLA2's alpha. Arguments as for forward(); every tensor on the GPU."""
+    import torch
+
+    class _SLAFunction(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, q_, k_, v_, w_, a_):
+            B, H, Np, d = q_.shape
+            n = Np if N is None else int(N)
+            p = make_params(B, H, n, d, variant=variant, k_crit=k_crit, k_neg=k_neg,
+                            softmax_scale=softmax_scale, w_proj=w_, proj_q=proj_q, proj_k=proj_k, alpha=a_,
+                            phi=phi)
+            q_, k_, v_ = q_.contiguous(), k_.contiguous(), v_.contiguous()
+            out, saved, ws = forward_train(q_, k_, v_, params=p)
+            ctx.p, ctx.saved, ctx.ws = p, saved, ws
+            ctx.save_for_backward(q_, k_, v_, w_, a_)
+            return out
+
+        @staticmethod
+        def backward(ctx, do):
+            q_, k_, v_, w_, a_ = ctx.saved_tensors
+            dq, dk, dv, pg, _ = backward(q_, k_, v_, do.contiguous(), params=ctx.p, saved=ctx.saved,
+                                         fwd_workspace=ctx.ws)
+            dw = pg.to(w_.dtype) if (w_ is not None and variant == "sla" and ctx.needs_input_grad[3]) else None
+            da = pg if (a_ is not None and variant == "sla2" and ctx.needs_input_grad[4]) else None
+            return dq, dk, dv, dw, da
+
+    return _SLAFunction.apply(q, k, v, w_proj, alpha)

@@ -189,3 +189,24 @@ def test_backward_full_size(cuda_lib, name, record_property):
     res = run_train(cuda_lib, inp, dO_bits)
     assert cuda_lib.read_device_status(res["fws"]) == 0
     check_head(res, inp, 5, dO_bits, record=record_property)
+
+
+def test_autograd_function_matches_sla_backward(cuda_lib):
+    """attention() through torch.autograd gives sla_backward's gradients, bit for bit."""
+    import torch
+
+    w = W.make_workload("bw_autograd", 1, 2, 64 * 6 + 9, 64, "sla2", k_crit=2, k_neg=0, seed=53)
+    inp = W.make_inputs(w)
+    dO_bits = W.grad_output(w)
+    res = run_train(cuda_lib, inp, dO_bits)
+    dev = res["dev"]
+    q, k, v = (dev[x].clone().requires_grad_(True) for x in ("q", "k", "v"))
+    alpha = dev["alpha"].clone().requires_grad_(True)
+    o = cuda_lib.attention(q, k, v, N=w.N, variant="sla2", k_crit=w.k_crit, alpha=alpha,
+                           proj_q=dev["proj_q"], proj_k=dev["proj_k"])
+    assert torch.equal(o.view(torch.int16)[:, :, :w.N], res["O"].view(torch.int16)[:, :, :w.N])
+    o.backward(res["do"])
+    torch.cuda.synchronize()
+    for t, ref in ((q, res["dq"]), (k, res["dk"]), (v, res["dv"])):
+        assert torch.equal(t.grad.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(alpha.grad, res["pg"])
