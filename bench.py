@@ -98,6 +98,52 @@ def backward_flops(w):
     return sparse + linear + proj
 
 
+# Shared-memory fill from L2 with every SM loading at once: 49 B per SM cycle,
+# measured with a standalone microbenchmark (TMA tensor loads of random
+# 64-row bf16 blocks from an L2-resident 16 MB source, 2-3 steps in flight, all
+# 148 SMs; cp.async reached 37.5 and the two paths together 29.6, so they share
+# one limit). The attention kernel's tile traffic is set against it.
+L2_FILL_B_PER_CYCLE_SM = 49.0
+
+
+def attention_tile_bytes(w):
+    """Bytes one bf16 attention launch moves from L2 into shared memory, from
+    its load schedule. Per CTA (two query blocks): the Q pair; per critical
+    step the K and V pairs, with phi(K)'s pair too when the excluded blocks'
+    products run in phase 1 (d = 128 with a linear branch); per phase-2 step
+    the phi(K) and V pairs (the negligible blocks, or at d = 64 every excluded
+    block); the phi(Q) pair when it is precomputed; SLA's W. None for the
+    quantised branch."""
+    if w.precision != "bf16":
+        return None
+    tile = 64 * w.d * 2
+    linear = w.k_crit + w.k_neg < w.Nb
+    merged = linear and w.d == 128
+    pre = linear and w.k_neg * 1260 < (w.k_crit + w.k_neg) * 350 + 8000
+    tiles = 2 + w.k_crit * (6 if merged else 4)
+    if linear:
+        tiles += 4 * (w.k_neg if merged else w.k_crit + w.k_neg)
+    if pre:
+        tiles += 2
+    extra = w.d * w.d * 2 if (w.variant == "sla" and linear) else 0
+    ctas = w.B * w.H * ((w.Nb + 1) // 2)
+    return ctas * (tiles * tile + extra)
+
+
+def l2_fill(w, attn_ms, clk, n_sm):
+    """The attention kernel's tile traffic per SM cycle (at the sampled median
+    SM clock) against the measured fill limit."""
+    tb = attention_tile_bytes(w)
+    if tb is None:
+        return None
+    mhz = clk.get("sm_mhz") if clk else None
+    per = tb / (attn_ms * 1e-3 * mhz * 1e6 * n_sm) if mhz else None
+    return {"tile_bytes": tb, "TB/s": round(tb / (attn_ms * 1e-3) / 1e12, 2), "sm_mhz": mhz,
+            "B_per_cycle_per_SM": None if per is None else round(per, 1),
+            "limit_B_per_cycle_per_SM": L2_FILL_B_PER_CYCLE_SM,
+            "frac": None if per is None else round(per / L2_FILL_B_PER_CYCLE_SM, 3)}
+
+
 def correction_flops(w):
     """Extra tensor FLOPs executed for H_i = H_tot - sum over excluded blocks."""
     return w.B * w.H * w.Nb * (w.k_crit + w.k_neg) * 4.0 * 64 * 64 * w.d
@@ -534,6 +580,12 @@ def run_ours(args):
            # pool, scores, classify, phi(K)/h/z, reduce, [Z_i,] attention
            "gpu_launches": (7 if w.k_crit + w.k_neg < w.Nb else 6) * args.steps,
            "clocks": clk}
+    import torch
+
+    n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    fill = l2_fill(w, attn_ms, clk, n_sm)
+    if fill is not None:
+        res["attention_l2_fill"] = fill
 
     if not args.no_backward and rank == 0 and w.precision == "bf16":
         bms, fms, dms = time_backward(sla, w, dev, 10, 2)
@@ -554,10 +606,12 @@ def run_ours(args):
         dev97 = device_inputs(inp97)
         ms97, st97, _ = time_forward(sla, w97, dev97, args.steps, args.warmup, 1, stage_timing=True)
         ms97 /= args.steps
+        fill97 = l2_fill(w97, st97["attention"], clk, n_sm)
         entry = {"workload": w97.name, "ms": round(ms97, 4),
                  "dense_eq_tflops": round(dense_eq_flops(w97) / (ms97 * 1e-3) / 1e12, 2),
                  "attention_ms": round(st97["attention"], 4),
-                 "attention_tflops": round(attention_flops(w97) / (st97["attention"] * 1e-3) / 1e12, 2)}
+                 "attention_tflops": round(attention_flops(w97) / (st97["attention"] * 1e-3) / 1e12, 2),
+                 "attention_l2_fill": fill97}
         if "dense_baseline" in res:
             entry["speedup_vs_dense"] = round(res["dense_baseline"]["ms"] / ms97, 3)
         entry["router_soft_topk"] = {"ms": round(time_router(sla, w97, dev97, 20, 3), 4), "tau": ROUTER_TAU,
