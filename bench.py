@@ -580,8 +580,6 @@ def run_ours(args):
            # pool, scores, classify, phi(K)/h/z, reduce, [Z_i,] attention
            "gpu_launches": (7 if w.k_crit + w.k_neg < w.Nb else 6) * args.steps,
            "clocks": clk}
-    import torch
-
     n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     fill = l2_fill(w, attn_ms, clk, n_sm)
     if fill is not None:
