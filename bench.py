@@ -41,9 +41,10 @@ SLA2_97_WORKLOAD = "sla2_b1h12n32768d128_s97"
 QUANT_WORKLOAD = "sla2_q_wan14b_b1h40n75600d128_s97"
 # dense tensor throughput of the 8-bit kinds relative to bf16 (2.25 vs 4.5 PFLOP/s nominal)
 LOWBIT_OVER_BF16 = 2.0
-# DRAM bytes (read + write) of one attention launch, from the ncu capture
-# summarised in profiles/attn_tc_kernel_sla_wan13b_b1h12n32768d128.md; keyed by
-# workload and valid only for the attention kernel that capture was taken of
+# DRAM bytes (read + write) of one attention launch from an ncu capture of
+# this build's attention kernel (dram__bytes_read.sum + dram__bytes_write.sum),
+# keyed by workload; a workload without a capture of the current kernel gets
+# null
 ATTN_TRAFFIC = {"sla_wan13b_b1h12n32768d128_s95": 421516288 + 91559424}
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "ms/forward and dense-equiv TFLOPS at 95-97% sparsity; tensor-pipe % of B200 peak"
@@ -61,7 +62,7 @@ def peaks():
 
 
 # ---------------------------------------------------------------------------
-# work accounting (algorithmic FLOPs / bytes; stated in the design doc)
+# work accounting (algorithmic FLOPs / bytes)
 # ---------------------------------------------------------------------------
 
 def dense_eq_flops(w):
@@ -145,8 +146,39 @@ def l2_fill(w, attn_ms, clk, n_sm):
 
 
 def correction_flops(w):
-    """Extra tensor FLOPs executed for H_i = H_tot - sum over excluded blocks."""
-    return w.B * w.H * w.Nb * (w.k_crit + w.k_neg) * 4.0 * 64 * 64 * w.d
+    """Tensor FLOPs of the complement G_i = sum over the excluded blocks of
+    phi(K_j)^T V_j (2 x 64 x d^2 per excluded block of each query block), which
+    forms H_i = H_tot - G_i; zero without a marginal block."""
+    if w.k_crit + w.k_neg >= w.Nb:
+        return 0.0
+    return w.B * w.H * w.Nb * (w.k_crit + w.k_neg) * 2.0 * 64 * w.d * w.d
+
+
+def useful_flops(w):
+    """Tensor FLOPs the attention kernel issues, less the masked parts of its
+    pair tiles (the off-diagonal quarters of S, the zero halves of P, the
+    discarded half of each phi(Q) H product): the algorithmic products plus
+    the complement G_i that forms H_i."""
+    return attention_flops(w) + correction_flops(w)
+
+
+def forward_launches(w):
+    """Kernels one sla_forward launches: pool, scores, classify, phi(K)/h/z,
+    the H_tot / Z_tot reduction, the attention kernel, and the Z_i kernel when
+    phi(Q) and Z_i are precomputed (a linear branch whose phase 2 is too short
+    to hide them, or the quantised branch)."""
+    linear = w.k_crit + w.k_neg < w.Nb
+    pre = linear and (w.precision != "bf16" or w.k_neg * 1260 < (w.k_crit + w.k_neg) * 350 + 8000)
+    return 7 if pre else 6
+
+
+def attention_peak(pk, pk_kind, timed_ms):
+    """bf16 tensor peak for the attention kernel: the burst figure when the
+    timed region lasts under two seconds (the clocks stay at their burst
+    level), the sustained figure for longer regions."""
+    if timed_ms < 2000.0:
+        return pk["bf16_tflops"], f"{pk_kind} bf16 burst (timed region {timed_ms / 1e3:.2f} s)"
+    return pk["bf16_tflops_sustained"], f"{pk_kind} bf16 sustained (timed region {timed_ms / 1e3:.2f} s)"
 
 
 def executed_flops(w):
@@ -546,8 +578,7 @@ def run_ours(args):
     attn_ms = stages["attention"]
     attn_alg = attention_flops(w)
     attn_tf = attn_alg / (attn_ms * 1e-3) / 1e12
-    peak_tf = pk["bf16_tflops_sustained"]
-    peak_kind = f"{pk_kind} bf16 sustained"
+    peak_tf, peak_kind = attention_peak(pk, pk_kind, ms_total)
     if w.precision != "bf16":
         # the INT8 / e4m3 sparse products run at the 8-bit rate, the rest at bf16
         f_lowbit, f_bf16 = attention_split_flops(w)
@@ -556,7 +587,10 @@ def run_ours(args):
     roofline = {"bound": "tensor", "achieved": round(attn_tf, 2), "peak": peak_tf,
                 "unit": "TFLOP/s", "frac": round(attn_tf / peak_tf, 4),
                 "traffic": ATTN_TRAFFIC.get(w.name), "kernel": "attention", "peak_kind": peak_kind,
-                "executed_tflops": round(executed_flops(w) / (attn_ms * 1e-3) / 1e12, 2)}
+                "launch_ms": round(attn_ms, 4),
+                "executed_excl_masked_tflops": round(useful_flops(w) / (attn_ms * 1e-3) / 1e12, 2),
+                "executed_excl_masked_frac": round(useful_flops(w) / (attn_ms * 1e-3) / 1e12 / peak_tf, 4),
+                "issued_tflops": round(executed_flops(w) / (attn_ms * 1e-3) / 1e12, 2)}
     in_bytes = 3 * w.B * w.H * w.N_pad * w.d * 2
     sb = stage_bytes(w)
     hbm = {k: {"ms": round(stages[k], 4), "GB/s": round(b / (stages[k] * 1e-3) / 1e9, 1),
@@ -577,8 +611,7 @@ def run_ours(args):
            "roofline": roofline,
            "stages_ms": {k: round(v, 4) for k, v in stages.items()},
            "hbm_stages": hbm,
-           # pool, scores, classify, phi(K)/h/z, reduce, [Z_i,] attention
-           "gpu_launches": (7 if w.k_crit + w.k_neg < w.Nb else 6) * args.steps,
+           "gpu_launches": forward_launches(w) * args.steps,
            "clocks": clk}
     n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     fill = l2_fill(w, attn_ms, clk, n_sm)
@@ -605,10 +638,16 @@ def run_ours(args):
         ms97, st97, _ = time_forward(sla, w97, dev97, args.steps, args.warmup, 1, stage_timing=True)
         ms97 /= args.steps
         fill97 = l2_fill(w97, st97["attention"], clk, n_sm)
+        t97 = st97["attention"] * 1e-3
+        pk97, pk97_kind = attention_peak(pk, pk_kind, ms97 * args.steps)
         entry = {"workload": w97.name, "ms": round(ms97, 4),
                  "dense_eq_tflops": round(dense_eq_flops(w97) / (ms97 * 1e-3) / 1e12, 2),
                  "attention_ms": round(st97["attention"], 4),
-                 "attention_tflops": round(attention_flops(w97) / (st97["attention"] * 1e-3) / 1e12, 2),
+                 "attention_tflops": round(attention_flops(w97) / t97 / 1e12, 2),
+                 "executed_excl_masked_tflops": round(useful_flops(w97) / t97 / 1e12, 2),
+                 "executed_excl_masked_frac": round(useful_flops(w97) / t97 / 1e12 / pk97, 4),
+                 "issued_tflops": round(executed_flops(w97) / t97 / 1e12, 2),
+                 "peak": pk97, "peak_kind": pk97_kind,
                  "attention_l2_fill": fill97}
         if "dense_baseline" in res:
             entry["speedup_vs_dense"] = round(res["dense_baseline"]["ms"] / ms97, 3)

@@ -64,7 +64,8 @@
 extern "C" {
 #endif
 
-#define SLA_ABI_VERSION 4 /* 2: sla_params.phi; 3: sla_router_soft_topk; 4: training forward, backward */
+#define SLA_ABI_VERSION 5 /* 2: sla_params.phi; 3: sla_router_soft_topk; 4: training forward, backward;
+                             5: sla_forward_noalloc, sla_read_device_status(NULL), sla_check_wait_timeout */
 #define SLA_BLOCK 64
 #define SLA_MAX_BLOCKS 4096 /* N <= 262144 */
 
@@ -236,8 +237,25 @@ sla_status sla_router_soft_topk(const void* Q, const void* K, const sla_params* 
 /* Synchronises the stream, then reads the device status word written by the
  * last sla_forward() on this workspace: SLA_OK, SLA_ERR_DEVICE_TIMEOUT if a
  * bounded in-kernel wait gave up, or SLA_ERR_DEVICE_CHECK if an in-kernel check
- * failed (in both cases the output is not valid). */
+ * failed (in both cases the output is not valid). workspace = NULL reads the
+ * status word of the last sla_forward_noalloc() on the current device. */
 sla_status sla_read_device_status(const void* workspace, void* stream);
+
+/* Failure-detection self-test (no counterpart on the pages). Every wait of the
+ * library's kernels on an mbarrier is bounded: when it expires, the kernel
+ * writes SLA_ERR_DEVICE_TIMEOUT's code into the workspace's status word and
+ * returns instead of hanging. This call makes exactly that happen, harmlessly:
+ * one thread waits, with the same wait routine, on an mbarrier that nothing
+ * arrives on, giving up after limit_cycles SM cycles (1 .. 4e9; the forward's
+ * kernels use 4e9, about 2 s). Nothing else is in flight, so the kernel returns
+ * normally and the context stays usable. Afterwards sla_read_device_status()
+ * on the same workspace returns SLA_ERR_DEVICE_TIMEOUT; the next sla_forward()
+ * on it clears the word.
+ *   workspace  device buffer of at least 256 bytes, 256-byte aligned (a forward
+ *              workspace may be used; only its status word is touched).
+ * Errors: SLA_ERR_WORKSPACE, SLA_ERR_INVALID_ARG for a limit out of range. */
+sla_status sla_check_wait_timeout(void* workspace, size_t workspace_bytes, long long limit_cycles,
+                                  void* stream);
 
 /* Dense softmax attention O = softmax(Q K^T * scale) V over all N keys, with
  * the same kernel machinery as the sparse branch (every block critical, no
@@ -268,8 +286,11 @@ sla_status sla_dense_forward(const void* Q, const void* K, const void* V, void* 
  *     GPU work overlaps (different streams, different host threads without
  *     ordering) race on the array and give undefined results: order them on
  *     one stream or serialise them.
- *   - The mask, lists and device status of these calls live in the shared
- *     array and are not readable through sla_get_mask / sla_read_device_status. */
+ *   - The mask and lists of these calls live in the shared array and are not
+ *     readable through sla_get_mask. Their device status word is: pass NULL as
+ *     the workspace of sla_read_device_status. A bounded in-kernel wait that
+ *     expires in a no-alloc call (SLA_ERR_DEVICE_TIMEOUT, output not valid) is
+ *     reported only there: the call itself has already returned SLA_OK. */
 #define SLA_NOALLOC_WORKSPACE_BYTES (32u << 20)
 sla_status sla_forward_noalloc(const void* Q, const void* K, const void* V, void* O,
                                const sla_params* p, void* stream);

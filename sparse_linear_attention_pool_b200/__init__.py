@@ -39,7 +39,7 @@ EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate", "sla_workspac
            "sla_forward", "sla_get_mask", "sla_get_pooled", "sla_read_device_status",
            "sla_dense_forward", "sla_stage_timing", "sla_stage_times", "sla_forward_noalloc",
            "sla_get_quantized", "sla_router_soft_topk", "sla_forward_train", "sla_backward_workspace_size",
-           "sla_backward")
+           "sla_backward", "sla_check_wait_timeout")
 NOALLOC_WORKSPACE_BYTES = 32 << 20
 NUM_STAGES = 6
 STAGES = ("pool", "scores", "classify", "phik_hz", "hz_reduce", "attention")
@@ -100,6 +100,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "sla_forward_train": (i, [vp, vp, vp, vp, P, ctypes.POINTER(Saved), vp, sz, vp]),
         "sla_backward_workspace_size": (sz, [P]),
         "sla_backward": (i, [vp, vp, vp, vp, P, ctypes.POINTER(Saved), vp, sz, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "sla_check_wait_timeout": (i, [vp, sz, ctypes.c_longlong, vp]),
         "sla_stage_timing": (i, [i]),
         "sla_stage_times": (i, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
     }
@@ -214,7 +215,15 @@ def get_pooled(p: Params, workspace, stream=None):
 
 
 def read_device_status(workspace, stream=None) -> int:
+    """Status word of the last forward on `workspace` (None: the last
+    sla_forward_noalloc on the current device); syncs the stream."""
     return load().sla_read_device_status(_ptr(workspace), _stream(stream))
+
+
+def check_wait_timeout(workspace, limit_cycles: int, stream=None) -> int:
+    """sla_check_wait_timeout: one bounded in-kernel wait that nothing ends,
+    given up after limit_cycles; its status lands in the workspace's status word."""
+    return load().sla_check_wait_timeout(_ptr(workspace), workspace.numel(), int(limit_cycles), _stream(stream))
 
 
 def dense_forward(q, k, v, *, N: Optional[int] = None, softmax_scale: float = 0.0, out=None,

@@ -257,10 +257,33 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     // bytes per ring step; dense mode loads one shared tile per step, the
     // quantised phase 1 one 8 KB code tile per block
     const int tileBytes = dense ? C::kTile : 2 * C::kTile;
+    // Abort safety: a copy is issued only after its slot's release was
+    // observed with no abort raised, so every slot has at most one copy in
+    // flight; once a wait fails or the abort flag is up, no further copy is
+    // issued. Before the warp leaves it waits (bounded, ignoring the abort
+    // flag) for the last copy of every slot it filled, so no TMA write to
+    // shared memory is still pending when the CTA exits.
+    bool stop = false;
+    auto pwait = [&](int b, uint32_t parity) {
+      const bool ok = !stop && wait(b, parity) && *abort_flag == 0;
+      stop = !__all_sync(0xffffffffu, ok);
+      return !stop;
+    };
+    uint32_t kpar = 0, kany = 0;  // per K slot: parity of its next fill; slots filled at least once
+    uint32_t vpar = 0, vany = 0;  // same for the V slots
+    auto k_filled = [&](int st) {
+      kany |= 1u << st;
+      kpar ^= 1u << st;
+    };
+    auto v_filled = [&](int st) {
+      vany |= 1u << st;
+      vpar ^= 1u << st;
+    };
     // phi(Q) (precomputed) over the Q or Q-code tiles once the last S product
     // has read them: the epilogue's phi(Q) H_i and phi(Q) Z_i operand
+    bool phiq_issued = false;
     auto load_phiq = [&]() {
-      wait(bQFree, 0);
+      if (!pwait(bQFree, 0)) return;
       if (lane == 0) {
         mbar_expect_tx(bar(bPhiQFull), 2 * C::kTile);
         for (int s = 0; s < C::kSub; ++s) {
@@ -268,6 +291,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           tma_load_3d(sQ + s * C::kSubS + C::kHalf, &maps.phiq, bar(bPhiQFull), s * 64, iB * 64, bh);
         }
       }
+      phiq_issued = true;
       __syncwarp();
     };
     const int codeBytes = 2 * 8192;
@@ -275,7 +299,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     int kA_reg = 0, kB_reg = 0;           // indices of the current 32-step window (K side)
     int vA_reg = 0, vB_reg = 0;           // indices of the window the V side reads
     if (!merge) {
-      for (int T = 0; T < nTot + lag; ++T) {
+      for (int T = 0; T < nTot + lag && !stop; ++T) {
         const int TK = T, TV = T - lag;
         if ((TK & 31) == 0 && TK < nTot) {
           const int Ti = TK + lane;
@@ -291,7 +315,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           const int jA = __shfl_sync(0xffffffffu, kA_reg, TK & 31);
           const int jB = __shfl_sync(0xffffffffu, kB_reg, TK & 31);
           const int st = TK % C::kNK;
-          wait(bKEmpty0 + st, ((TK / C::kNK) & 1) ^ 1);
+          if (!pwait(bKEmpty0 + st, ((TK / C::kNK) & 1) ^ 1)) break;
           if (lane == 0) {
             const uint32_t slot = sK + st * C::kPair;
             if (QNT && TK < nA) {
@@ -308,13 +332,14 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
               }
             }
           }
+          k_filled(st);
           __syncwarp();
         }
         if (TV >= 0 && TV < nTot) {
           const int jA = __shfl_sync(0xffffffffu, vA_reg, TV & 31);
           const int jB = __shfl_sync(0xffffffffu, vB_reg, TV & 31);
           const int st = TV % C::kNV;
-          wait(bVEmpty0 + st, ((TV / C::kNV) & 1) ^ 1);
+          if (!pwait(bVEmpty0 + st, ((TV / C::kNV) & 1) ^ 1)) break;
           if (lane == 0) {
             const uint32_t slot = sV + st * C::kPair;
             if (QNT && TV < nA) {
@@ -330,6 +355,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
               }
             }
           }
+          v_filled(st);
           __syncwarp();
         }
       }
@@ -347,7 +373,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       };
       uint32_t pe = (1u << C::kNK) - 1;  // KEmpty parity per slot (a slot's first fill passes)
       uint32_t pd = 0;                   // KDone parity per slot
-      for (int t = 0; t <= nA; ++t) {
+      for (int t = 0; t <= nA && !stop; ++t) {
         if ((t & 31) == 0 && t < nA) {
           const int Ti = t + lane;
           kA_reg = Ti < nA ? step_block(0, Ti) : 0;
@@ -362,9 +388,10 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           const int jA = __shfl_sync(0xffffffffu, kA_reg, t & 31);
           const int jB = __shfl_sync(0xffffffffu, kB_reg, t & 31);
           const int st = t % C::kNK;
-          wait(bKEmpty0 + st, (pe >> st) & 1u);
+          if (!pwait(bKEmpty0 + st, (pe >> st) & 1u)) break;
           pe ^= 1u << st;
           if (lane == 0) load_pair(sK + st * C::kPair, &maps.k, bar(bKFull0 + st), jA, jB);
+          k_filled(st);
           __syncwarp();
         }
         if (t >= 1) {  // V(t-1), then phi(K)(t-1)
@@ -372,17 +399,19 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           const int jA = __shfl_sync(0xffffffffu, vA_reg, u & 31);
           const int jB = __shfl_sync(0xffffffffu, vB_reg, u & 31);
           const int sv = u % C::kNV, st = u % C::kNK;
-          wait(bVEmpty0 + sv, ((u / C::kNV) & 1) ^ 1);
+          if (!pwait(bVEmpty0 + sv, ((u / C::kNV) & 1) ^ 1)) break;
           if (lane == 0) load_pair(sV + sv * C::kPair, &maps.v, bar(bVFull0 + sv), jA, jB);
+          v_filled(sv);
           __syncwarp();
-          wait(bKDone0 + st, (pd >> st) & 1u);
+          if (!pwait(bKDone0 + st, (pd >> st) & 1u)) break;
           pd ^= 1u << st;
           if (lane == 0) load_pair(sK + st * C::kPair, &maps.phik, bar(bKFull0 + st), jA, jB);
+          k_filled(st);
           __syncwarp();
         }
       }
-      if (pre) load_phiq();  // S(nA-1) has completed: phi(K)(nA-1) waited for it
-      for (int u = 0; u < nP2; ++u) {  // the negligible blocks
+      if (pre && !stop) load_phiq();  // S(nA-1) has completed: phi(K)(nA-1) waited for it
+      for (int u = 0; u < nP2 && !stop; ++u) {  // the negligible blocks
         const int T = nA + u;
         if ((u & 31) == 0) {
           const int Ti = T + lane;
@@ -392,23 +421,37 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         const int jA = __shfl_sync(0xffffffffu, kA_reg, u & 31);
         const int jB = __shfl_sync(0xffffffffu, kB_reg, u & 31);
         const int st = T % C::kNK, sv = T % C::kNV;
-        wait(bKEmpty0 + st, (pe >> st) & 1u);
+        if (!pwait(bKEmpty0 + st, (pe >> st) & 1u)) break;
         pe ^= 1u << st;
         if (lane == 0) load_pair(sK + st * C::kPair, &maps.phik, bar(bKFull0 + st), jA, jB);
+        k_filled(st);
         __syncwarp();
-        wait(bVEmpty0 + sv, ((T / C::kNV) & 1) ^ 1);
+        if (!pwait(bVEmpty0 + sv, ((T / C::kNV) & 1) ^ 1)) break;
         if (lane == 0) load_pair(sV + sv * C::kPair, &maps.v, bar(bVFull0 + sv), jA, jB);
+        v_filled(sv);
         __syncwarp();
       }
     }
-    if (pre && !merge) load_phiq();
-    if (use_y && lane == 0) {  // W reuses the rings once every loop product has completed
-      wait(bTailDone, 0);
-      mbar_expect_tx(bar(bWFull), C::kMat);
-      for (int s = 0; s < C::kSub; ++s) tma_load_2d(sW + s * (D * 128), &maps.w, bar(bWFull), s * 64, 0);
-      wait_drain(bWFull, 0);  // leave only after the copies have landed
+    if (pre && !merge && !stop) load_phiq();
+    bool w_issued = false;
+    if (use_y && pwait(bTailDone, 0)) {  // W reuses the rings once every loop product has completed
+      if (lane == 0) {
+        mbar_expect_tx(bar(bWFull), C::kMat);
+        for (int s = 0; s < C::kSub; ++s) tma_load_2d(sW + s * (D * 128), &maps.w, bar(bWFull), s * 64, 0);
+      }
+      w_issued = true;
     }
-    if (lane == 0 && pre) wait_drain(bPhiQFull, 0);
+    // drain: the last copy of every slot, Q, phi(Q) and W have landed
+    if (lane == 0) {
+      wait_drain(bQFull, 0);
+      for (int st = 0; st < C::kNK; ++st)
+        if ((kany >> st) & 1u) wait_drain(bKFull0 + st, ((kpar >> st) & 1u) ^ 1u);
+      for (int st = 0; st < C::kNV; ++st)
+        if ((vany >> st) & 1u) wait_drain(bVFull0 + st, ((vpar >> st) & 1u) ^ 1u);
+      if (phiq_issued) wait_drain(bPhiQFull, 0);
+      if (w_issued) wait_drain(bWFull, 0);
+    }
+    __syncwarp();
   } else if (warp == 5) {
     // ------------------------------ MMA issuer ------------------------------
     // The whole warp walks the loop (warp-uniform descriptors); the MMA and

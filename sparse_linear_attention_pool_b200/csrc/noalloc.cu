@@ -11,7 +11,8 @@
 // library and stays resident until the process exits. Kernels need its device
 // address, which host code obtains with cudaGetSymbolAddress (the array's name
 // in host code is only a host-side stand-in); that lookup runs once per device,
-// with that device current, on the first call made on it.
+// with that device current, on the first call made on it (or on the first
+// sla_read_device_status(NULL, ...) there).
 #include <mutex>
 
 #include "sla_internal.cuh"
@@ -24,8 +25,12 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 void* g_dev_ptr[kMaxDevices] = {};
 
+}  // namespace
+
+namespace sla {
+
 // Device address of the static workspace on the current device (looked up once).
-sla_status workspace_address(void** out) {
+sla_status noalloc_workspace_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return SLA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SLA_ERR_UNSUPPORTED;
@@ -40,7 +45,7 @@ sla_status workspace_address(void** out) {
   return SLA_OK;
 }
 
-}  // namespace
+}  // namespace sla
 
 extern "C" sla_status sla_forward_noalloc(const void* Q, const void* K, const void* V, void* O,
                                           const sla_params* p, void* stream) {
@@ -48,7 +53,7 @@ extern "C" sla_status sla_forward_noalloc(const void* Q, const void* K, const vo
   if (st != SLA_OK) return st;
   if (sla_workspace_size(p) > size_t(SLA_NOALLOC_WORKSPACE_BYTES)) return SLA_ERR_WORKSPACE;
   void* ws = nullptr;
-  const sla_status ws_st = workspace_address(&ws);
+  const sla_status ws_st = sla::noalloc_workspace_address(&ws);
   if (ws_st != SLA_OK) return ws_st;
   // sla_forward clears the part of the workspace that must start at zero (the
   // device status word) and overwrites everything else it reads.

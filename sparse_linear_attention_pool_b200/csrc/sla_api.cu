@@ -400,7 +400,13 @@ sla_status sla_get_quantized(const sla_params* p, const void* workspace, int8_t*
 }
 
 sla_status sla_read_device_status(const void* workspace, void* stream) {
-  if (workspace == nullptr || !aligned(workspace, 256)) return SLA_ERR_WORKSPACE;
+  if (workspace == nullptr) {  // the no-alloc entry point's static workspace on this device
+    void* ws = nullptr;
+    const sla_status st = noalloc_workspace_address(&ws);
+    if (st != SLA_OK) return st;
+    workspace = ws;
+  }
+  if (!aligned(workspace, 256)) return SLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int word = 0;
   cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);

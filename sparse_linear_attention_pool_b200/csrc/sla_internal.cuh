@@ -17,6 +17,10 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Status-word codes written by kernels into the first bytes of the workspace.
 enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1, kDevBadIndex = 2 };
 
+// Device address of sla_forward_noalloc's static workspace on the current
+// device (looked up once per device; defined in noalloc.cu).
+sla_status noalloc_workspace_address(void** out);
+
 // Tokens per CTA in the phi(K) / h / z pass (8 blocks).
 constexpr int kHzChunk = 512;
 

@@ -48,22 +48,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of `bar` with the given parity to complete.
-// Gives up after ~kWaitCycles SM cycles (about 2 s): records the timeout in
-// the device status word and in the CTA's abort flag, and returns false.
-constexpr long long kWaitCycles = 4000000000LL;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+// Gives up after `limit` SM cycles: records the timeout in the device status
+// word and in the CTA's abort flag, and returns false. A set abort flag makes
+// the wait return false at once.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                              int* status, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       if (status) atomicExch(status, kDevTimeout);
       return false;
     }
   }
+}
+// The kernels' waits: about 2 s at the B200's clocks.
+constexpr long long kWaitCycles = 4000000000LL;
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+  return mbar_wait_for(bar, parity, abort_flag, status, kWaitCycles);
 }
 
 // ---- TMA ----

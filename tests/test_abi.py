@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.sla_abi_version() == 4
+    assert lib.sla_abi_version() == 5
     for s in range(8):
         assert sla.status_string(s)
     assert "unknown" in sla.status_string(99)
@@ -124,7 +124,26 @@ def test_forward_rejects_on_host(lib):
     assert lib.sla_dense_forward(0x10000, 0x20000, 0x30000, 0x40000, 1, 1, 64, 80, 0.0, None) == \
         sla.SLA_ERR_UNSUPPORTED
     assert lib.sla_get_mask(ctypes.byref(p), None, None, None, None, None) == sla.SLA_ERR_WORKSPACE
-    assert lib.sla_read_device_status(None, None) == sla.SLA_ERR_WORKSPACE
+    assert lib.sla_read_device_status(0x50080, None) == sla.SLA_ERR_WORKSPACE  # not 256-aligned
+    # the bounded-wait self-test: a workspace of at least one 256-byte status block, a limit in range
+    assert lib.sla_check_wait_timeout(None, 256, 100000, None) == sla.SLA_ERR_WORKSPACE
+    assert lib.sla_check_wait_timeout(0x50080, 256, 100000, None) == sla.SLA_ERR_WORKSPACE
+    assert lib.sla_check_wait_timeout(0x50000, 255, 100000, None) == sla.SLA_ERR_WORKSPACE
+    assert lib.sla_check_wait_timeout(0x50000, 256, 0, None) == sla.SLA_ERR_INVALID_ARG
+    assert lib.sla_check_wait_timeout(0x50000, 256, 4000000001, None) == sla.SLA_ERR_INVALID_ARG
+
+
+def test_header_constants_match_the_binding():
+    text = open(os.path.join(ROOT, "include", "sla.h")).read()
+
+    def define(name):
+        m = re.search(r"#define\s+" + name + r"\s+(.+?)\s*(/\*.*)?$", text, flags=re.M)
+        assert m, name
+        return eval(m.group(1).replace("u", ""))  # plain integer expressions such as (32u << 20)
+
+    assert define("SLA_NOALLOC_WORKSPACE_BYTES") == sla.NOALLOC_WORKSPACE_BYTES
+    assert define("SLA_NUM_STAGES") == sla.NUM_STAGES == len(sla.STAGES)
+    assert define("SLA_BLOCK") == sla.BLOCK
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

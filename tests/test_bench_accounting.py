@@ -46,8 +46,35 @@ def test_linear_and_projection_terms():
     assert rest == pytest.approx(2 * (2.0 * BH * N * d * d), rel=1e-15)  # phi(Q) H and O^l W
     w2 = W.WORKLOADS["sla2_b1h12n32768d128_s97"]
     assert bench.attention_split_flops(w2)[1] == pytest.approx(2.0 * BH * N * d * d, rel=1e-15)
-    # the correction: one d x d x 64 product per excluded (query block, key block) pair
-    assert bench.correction_flops(w) == pytest.approx(BH * w.Nb * (w.k_crit + w.k_neg) * 4.0 * 64 * 64 * d)
+    # the correction: one d x 64 x d product per excluded (query block, key block) pair
+    assert bench.correction_flops(w) == pytest.approx(BH * w.Nb * (w.k_crit + w.k_neg) * 2.0 * 64 * d * d)
+    w64 = W.make_workload("c64", 1, 2, 64 * 20, 64, "sla", k_crit=2, k_neg=3, seed=0)
+    assert bench.correction_flops(w64) == pytest.approx(2 * 20 * 5 * 2.0 * 64 * 64 * 64)
+    assert bench.correction_flops(all_critical()) == 0.0  # no marginal block, no H_i
+
+
+def test_useful_work_of_the_sla2_97_workload():
+    # sparse pairs 12 heads x 512 blocks x 15 x 4 x 64 x 64 x 128 = 1.933e11, the
+    # complement as much again (d = 128), phi(Q) H 2 N d^2 per head = 1.29e10
+    w = W.WORKLOADS["sla2_b1h12n32768d128_s97"]
+    sparse = 12 * 512 * 15 * 4.0 * 64 * 64 * 128
+    assert bench.useful_flops(w) == pytest.approx(2 * sparse + 12 * 2.0 * 32768 * 128 * 128, rel=1e-12)
+    # issued work adds the masked halves: the sparse pairs and phi(Q) H twice, the complement once
+    assert bench.executed_flops(w) == pytest.approx(3 * sparse + 2 * 12 * 2.0 * 32768 * 128 * 128, rel=1e-12)
+
+
+def test_launch_count_per_forward():
+    # pool, scores, classify, phi(K)/h/z, reduction, attention; + Z_i when precomputed
+    assert bench.forward_launches(W.WORKLOADS["sla_wan13b_b1h12n32768d128_s95"]) == 6  # 51 negligible
+    assert bench.forward_launches(W.WORKLOADS["sla2_b1h12n32768d128_s97"]) == 7
+    assert bench.forward_launches(W.WORKLOADS["sla2_q_wan14b_b1h40n75600d128_s97"]) == 7
+    assert bench.forward_launches(all_critical()) == 6  # no linear branch
+
+
+def test_peak_choice_follows_the_timed_region():
+    pk = {"bf16_tflops": 1672.7, "bf16_tflops_sustained": 1414.8}
+    assert bench.attention_peak(pk, "measured", 35.0)[0] == 1672.7
+    assert bench.attention_peak(pk, "measured", 5000.0)[0] == 1414.8
 
 
 def test_job_value_counts_every_rank():
