@@ -24,7 +24,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import tempfile
 import time
@@ -256,55 +255,90 @@ def stage_bytes(w):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of one GPU, sampled during the timed
+    region. NVML is polled from a host thread every ~2 ms (nvidia-smi's own
+    interval, 100 ms, is longer than a short timed region); the samples whose
+    host time falls between begin() and end() are summarised. Without NVML the
+    summary is None."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
     def __init__(self, device_index):
         self.idx = device_index
-        self.proc = None
-        # the sampled clock log (CSV) goes to $SLA_BENCH_LOG_DIR, else the temp directory
+        self.samples = []  # (host time, sm MHz, max sm MHz, reasons bitmask)
+        self.t0 = self.t1 = None
+        self.thread = None
         log_dir = os.environ.get("SLA_BENCH_LOG_DIR") or tempfile.gettempdir()
         self.path = os.path.join(log_dir, f"sla_bench_clocks_rank{device_index}.csv")
 
+    def _handle(self, nv):
+        import torch
+
+        try:  # the NVML device behind this CUDA device (CUDA_VISIBLE_DEVICES may renumber)
+            props = torch.cuda.get_device_properties(self.idx)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:  # noqa: BLE001
+            return nv.nvmlDeviceGetHandleByIndex(self.idx)
+
     def start(self):
+        import threading
+
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = self._handle(nv)
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001
+            self.thread = None
+            return
+        self.stop_flag = threading.Event()
+        first = threading.Event()
+
+        def run():
+            while not self.stop_flag.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:  # noqa: BLE001
+                    break
+                self.samples.append((time.perf_counter(), sm, mx, rs))
+                first.set()
+                time.sleep(0.002)
+            first.set()
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+        first.wait(timeout=5.0)
+
+    def begin(self):
+        self.t0 = time.perf_counter()
+
+    def end(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
+        self.stop_flag.set()
+        self.thread.join(timeout=5.0)
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            with open(self.path, "w") as f:
+                f.write("host_s,sm_mhz,sm_max_mhz,reasons_hex,in_timed_region\n")
+                for t, sm, mx, rs in self.samples:
+                    inside = self.t0 is not None and self.t0 <= t <= (self.t1 or t)
+                    f.write(f"{t:.6f},{sm},{mx},{rs:#x},{int(inside)}\n")
+        except OSError:
+            pass
+        inside = [x for x in self.samples if self.t0 is not None and self.t0 <= x[0] <= (self.t1 or x[0])]
+        if not inside:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = sorted({name for _, _, _, rs in inside for name, bit in self.REASONS if rs & bit})
+        return {"sm_mhz": statistics.median([x[1] for x in inside]), "sm_max_mhz": max(x[2] for x in inside),
+                "reasons": reasons, "samples": len(inside), "source": "nvml, ~2 ms interval"}
 
 
 # ---------------------------------------------------------------------------
@@ -391,11 +425,14 @@ def time_forward(sla, w, dev, steps, warmup, world, stage_timing=False, clocks=N
     torch.cuda.synchronize()
     if clocks:
         clocks.start()
+        clocks.begin()
     start.record(stream)
     for _ in range(steps):
         sla.forward(dev["q"], dev["k"], dev["v"], out=out, workspace=ws, params=p, stream=stream)
     end.record(stream)
     torch.cuda.synchronize()
+    if clocks:
+        clocks.end()
     barrier(world)
     clk = clocks.stop() if clocks else None
     ms = start.elapsed_time(end)

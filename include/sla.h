@@ -175,7 +175,10 @@ size_t sla_backward_workspace_size(const sla_params* p);
  *   dalpha        SLA2: [H] float32 device output, sum over the batch of
  *                 dO . (O^s - O^l); may be NULL. Must be NULL for SLA.
  *   workspace     at least sla_backward_workspace_size(p) bytes, 256-byte aligned.
- * bf16 precision only. The result is deterministic (no floating-point atomics). */
+ * bf16 precision only. The result is deterministic (no floating-point atomics).
+ * A bounded in-kernel wait that expires during the backward is recorded in
+ * the forward workspace's status word: check it with
+ * sla_read_device_status(fwd_workspace, stream). */
 sla_status sla_backward(const void* Q, const void* K, const void* V, const void* dO, const sla_params* p,
                         const sla_saved* saved, const void* fwd_workspace, size_t fwd_workspace_bytes, void* dQ,
                         void* dK, void* dV, float* dW, float* dalpha, void* workspace, size_t workspace_bytes,

@@ -534,10 +534,14 @@ def backward_f64(q, k, v, Mc, do, N, *, variant, scale, W=None, alpha_h=None, ph
 #   * S = (Qc Kc^T exact integer) * s_q * s_k * softmax_scale.
 #   * P~ = 2^(x - m) with x = S log2(e) and m = ceil(max_j x) the row max
 #     rounded up to an integer, so P~ is in (0, 1] and its largest entry in
-#     (1/2, 1]: the FP8 scale of a row of P is a power of two. A softmax of
-#     any max offset gives the same P / l; a power-of-two scale makes the e4m3
-#     codes of P independent of which integer offset a kernel holds when it
-#     quantises (a running max only shifts the exponent).
+#     (1/2, 1]. The pages fix only that P is scaled before the product and
+#     restored after; the scale of a row is taken as a power of two because
+#     e4m3 rounding commutes with multiplication by 2^k for values that stay
+#     normal and below the saturation bound: quantise(P 2^k) 2^-k is then the
+#     same value for every such k, so the scale adds no rounding of its own
+#     and the result does not depend on how the offset is reached. The offset
+#     puts the row's largest P~ in (1/2, 1], i.e. its code (after the 2^8
+#     multiplier below) in (128, 256], inside e4m3's normal range and below 448.
 #   * Each key block's V scale is folded into P relative to the largest V
 #     scale of the head, r_j = s_v,j / max_j s_v,j (one float32 division), and
 #     P enters the PV product as e4m3(P~ * r_j * 2^8); the row sum l uses the

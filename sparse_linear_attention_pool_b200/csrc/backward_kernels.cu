@@ -496,6 +496,7 @@ struct QArgs {
   const bf16* hblk;
   const float *ztot, *zblk;
   const float* alpha;  // SLA2 [H] (dO^s = alpha dO); null for SLA
+  const float* dQs;    // tcgen05 sparse partial (scaled); null: run the sparse loop here
   bf16* dQ;
   float scale, scale_log2;
   int H, N, Npad, Nb, kc, kn, phi_elu1;
@@ -537,7 +538,7 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(const QArgs a) {
     load_tile<D>(buf + T::kTile, a.V + headbase + size_t(j) * 64 * D, nvj);
     cp_async_commit();
   };
-  load_pair(0);
+  if (!a.dQs) load_pair(0);
   // H_i = H_tot - sum over the excluded blocks of h_j, Z_i likewise (while the
   // first tiles land)
   if (linear)
@@ -554,8 +555,9 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(const QArgs a) {
   float dq[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) dq[nt][0] = dq[nt][1] = dq[nt][2] = dq[nt][3] = 0.0f;
-  for (int t = 0; t < a.kc; ++t) {
-    if (t + 1 < a.kc) {
+  const int nsteps = a.dQs ? 0 : a.kc;
+  for (int t = 0; t < nsteps; ++t) {
+    if (t + 1 < nsteps) {
       load_pair(t + 1);
       cp_async_wait<1>();
     } else {
@@ -583,6 +585,7 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(const QArgs a) {
     mma_pz<NT, 2>(dq, s, Ks, T::LD, lane);
     __syncthreads();  // this buffer is refilled two pairs on
   }
+  cp_async_wait<0>();  // Q, dO, dnum landed even without a sparse pair (the barrier below publishes them)
   // the two key halves' partial dQ: the second half's warps hand theirs over
   // (rows D + 4 floats apart, so a fragment's eight rows fall in distinct banks)
   constexpr int RS = D + 4;
@@ -606,6 +609,22 @@ __global__ void __launch_bounds__(256, 1) bwd_q_kernel(const QArgs a) {
     dq[nt][1] = (dq[nt][1] + x0.y) * a.scale;
     dq[nt][2] = (dq[nt][2] + x1.x) * a.scale;
     dq[nt][3] = (dq[nt][3] + x1.y) * a.scale;
+  }
+  if (a.dQs) {  // the tcgen05 loop's partial (already scaled)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int c = nt * 8 + 2 * q;
+      if (va) {
+        const float2 x = *reinterpret_cast<const float2*>(a.dQs + (rowbase + ra) * D + c);
+        dq[nt][0] += x.x;
+        dq[nt][1] += x.y;
+      }
+      if (vb) {
+        const float2 x = *reinterpret_cast<const float2*>(a.dQs + (rowbase + rb) * D + c);
+        dq[nt][2] += x.x;
+        dq[nt][3] += x.y;
+      }
+    }
   }
 
   if (linear) {
@@ -646,6 +665,7 @@ struct KVArgs {
   const bf16* dhblk;
   const float *dztot, *dzblk;
   const float* alpha;  // SLA2 [H]; null for SLA
+  const float *dKs, *dVs;  // tcgen05 sparse partials (scaled); null: run the sparse loop here
   bf16 *dK, *dV;
   float scale, scale_log2;
   int H, N, Npad, Nb, linear, phi_elu1;
@@ -679,7 +699,7 @@ __global__ void __launch_bounds__(256, 1) bwd_kv_kernel(const KVArgs a) {
   load_tile<D>(Vs, a.V + rowbase * D, nvj);
   load_tile<D>(PKs, a.phik + rowbase * D, nvj);
   cp_async_commit();
-  const int nC = a.cntC[size_t(bh) * a.Nb + j];
+  const int nC = a.dKs ? 0 : a.cntC[size_t(bh) * a.Nb + j];
   const int* colC = a.colC + (size_t(bh) * a.Nb + j) * a.Nb;
   auto load_pair = [&](int t) {
     const int i = colC[t];
@@ -784,6 +804,22 @@ __global__ void __launch_bounds__(256, 1) bwd_kv_kernel(const KVArgs a) {
     dv[nt][2] = (dv[nt][2] + v1.x) * asc;
     dv[nt][3] = (dv[nt][3] + v1.y) * asc;
   }
+  if (a.dKs) {  // the sparse partials of the tcgen05 loop (already scaled); pad rows hold no data
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int c = nt * 8 + 2 * q;
+      if (va) {
+        const float2 k0 = *reinterpret_cast<const float2*>(a.dKs + (rowbase + ra) * D + c);
+        const float2 v0 = *reinterpret_cast<const float2*>(a.dVs + (rowbase + ra) * D + c);
+        dk[nt][0] += k0.x; dk[nt][1] += k0.y; dv[nt][0] += v0.x; dv[nt][1] += v0.y;
+      }
+      if (vb) {
+        const float2 k1 = *reinterpret_cast<const float2*>(a.dKs + (rowbase + rb) * D + c);
+        const float2 v1 = *reinterpret_cast<const float2*>(a.dVs + (rowbase + rb) * D + c);
+        dk[nt][2] += k1.x; dk[nt][3] += k1.y; dv[nt][2] += v1.x; dv[nt][3] += v1.y;
+      }
+    }
+  }
 
   if (a.linear) {
     mma_xz<NT, D>(dv, PKs, T::LD, r0, As, T::LD, lane);  // dV += phi(K_j) A_j
@@ -867,10 +903,17 @@ cudaError_t run_backward(const BwdArgs& a, cudaStream_t s) {
   }
   const float scale = a.scale;
   const float* alpha = a.sla ? nullptr : a.alpha;
-  // 5. dQ
+  // 5. dQ: at d = 128 the sparse loop on tcgen05 first (fp32 partial)
+  const bool tcq = D == 128 && a.dqs != nullptr;
+  if (e == cudaSuccess && tcq) {
+    QTcArgs ta{a.crit, a.save_lse, a.Drow, alpha, a.dqs, a.status, L.H, L.N, L.Npad, Nb, L.kc, scale,
+               scale * kLog2e};
+    e = launch_bwd_q_tc(a.Q, a.K, a.V, a.dO, ta, BH, s);
+  }
   if (e == cudaSuccess) {
     QArgs qa{a.Q, a.K, a.V, a.dO, a.dnum, a.crit, a.neg, a.save_lse, a.Drow, a.dden, a.htot, a.hblk, a.ztot,
-             a.zblk, alpha, a.dQ, scale, scale * kLog2e, L.H, L.N, L.Npad, Nb, L.kc, L.kn, a.phi_elu1};
+             a.zblk, alpha, tcq ? a.dqs : nullptr, a.dQ, scale, scale * kLog2e, L.H, L.N, L.Npad, Nb, L.kc, L.kn,
+             a.phi_elu1};
     const int bytes = (7 * T::kTile + T::kMat) * 2 + D * 4;
     e = set_smem(bwd_q_kernel<D>, bytes);
     if (e == cudaSuccess) {
@@ -878,11 +921,18 @@ cudaError_t run_backward(const BwdArgs& a, cudaStream_t s) {
       e = cudaGetLastError();
     }
   }
-  // 6. dK, dV
+  // 6. dK, dV: at d = 128 the sparse loop on tcgen05 first (fp32 partials)
+  // (the lse rows arrive by bulk copy: 16-byte aligned global addresses only)
+  const bool tc = D == 128 && a.dks != nullptr && (reinterpret_cast<uintptr_t>(a.save_lse) & 15) == 0;
+  if (e == cudaSuccess && tc) {
+    KvTcArgs ta{a.colC, a.cntC, a.save_lse, a.Drow, alpha, a.dks, a.dvs, a.status, L.H, L.N, L.Npad, Nb, scale,
+                scale * kLog2e};
+    e = launch_bwd_kv_tc(a.Q, a.K, a.V, a.dO, ta, BH, s);
+  }
   if (e == cudaSuccess) {
     KVArgs ka{a.Q, a.K, a.V, a.dO, a.phik, a.colC, a.colE, a.cntC, a.cntE, a.save_lse, a.Drow, a.dhtot,
-              a.dhblk, a.dztot, a.dzblk, alpha, a.dK, a.dV, scale, scale * kLog2e, L.H, L.N, L.Npad, Nb,
-              L.linear ? 1 : 0, a.phi_elu1};
+              a.dhblk, a.dztot, a.dzblk, alpha, tc ? a.dks : nullptr, tc ? a.dvs : nullptr, a.dK, a.dV, scale,
+              scale * kLog2e, L.H, L.N, L.Npad, Nb, L.linear ? 1 : 0, a.phi_elu1};
     const int bytes = (7 * T::kTile + T::kMat) * 2 + (D + 256) * 4;
     e = set_smem(bwd_kv_kernel<D>, bytes);
     if (e == cudaSuccess) {

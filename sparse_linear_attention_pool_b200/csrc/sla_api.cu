@@ -265,6 +265,10 @@ sla_status sla_backward(const void* Q, const void* K, const void* V, const void*
   a.colE = reinterpret_cast<int*>(ws + BL.cole);
   a.cntC = reinterpret_cast<int*>(ws + BL.cntc);
   a.cntE = reinterpret_cast<int*>(ws + BL.cnte);
+  a.dks = BL.d == 128 ? reinterpret_cast<float*>(ws + BL.dks) : nullptr;
+  a.dvs = BL.d == 128 ? reinterpret_cast<float*>(ws + BL.dvs) : nullptr;
+  a.dqs = BL.d == 128 ? reinterpret_cast<float*>(ws + BL.dqs) : nullptr;
+  a.status = reinterpret_cast<int*>(const_cast<unsigned char*>(fw) + L.status);
   a.dQ = static_cast<__nv_bfloat16*>(dQ);
   a.dK = static_cast<__nv_bfloat16*>(dK);
   a.dV = static_cast<__nv_bfloat16*>(dV);

@@ -150,7 +150,7 @@ cudaError_t launch_attention(const AttnArgs& a, int BH, int d, int mode, cudaStr
 struct BwLayout {
   int B, H, BH, N, Npad, Nb, d, kc, kn;
   bool linear, sla;
-  size_t dnum, phiq, drow, dden, dzblk, dztot, hblk, dhblk, dhtot, dwpart, dapart, colc, cole, cntc, cnte, total;
+  size_t dnum, phiq, drow, dden, dzblk, dztot, hblk, dhblk, dhtot, dwpart, dapart, colc, cole, cntc, cnte, dks, dvs, dqs, total;
 };
 
 inline BwLayout make_bw_layout(const sla_params& p) {
@@ -188,6 +188,9 @@ inline BwLayout make_bw_layout(const sla_params& p) {
   L.cole = take(BH * Nb * Nb * 4);
   L.cntc = take(BH * Nb * 4);
   L.cnte = take(BH * Nb * 4);
+  L.dks = take(d == 128 ? rows * d * 4 : 0);  // tcgen05 sparse partials (d = 128)
+  L.dvs = take(d == 128 ? rows * d * 4 : 0);
+  L.dqs = take(d == 128 ? rows * d * 4 : 0);
   L.total = off;
   return L;
 }
@@ -202,6 +205,8 @@ struct BwdArgs {
   float *Drow, *dden, *dzblk, *dztot, *dhtot, *dwpart, *dapart;
   __nv_bfloat16 *hblk, *dhblk;  // per-block d x d, read only by the complement sums
   int *colC, *colE, *cntC, *cntE;
+  float *dks, *dvs, *dqs;
+  int* status;
   __nv_bfloat16 *dQ, *dK, *dV;
   float *dW, *dalpha;
   float scale;
@@ -209,6 +214,35 @@ struct BwdArgs {
   int phi_elu1;
 };
 cudaError_t launch_backward(const BwdArgs& a, cudaStream_t s);
+
+// tcgen05 sparse loop of dK / dV (d = 128): fp32 partials, dK x scale, dV x asc
+struct KvTcArgs {
+  const int* colC;   // [BH][Nb][Nb]
+  const int* cntC;   // [BH][Nb]
+  const float* lse;  // [BH][Npad], natural log
+  const float* Drow; // [BH][Npad]
+  const float* alpha;
+  float* dKs;        // [BH][Npad][128]
+  float* dVs;
+  int* status;
+  int H, N, Npad, Nb;
+  float scale, scale_log2;
+};
+// tcgen05 sparse loop of dQ (d = 128): fp32 partial, x scale
+struct QTcArgs {
+  const int32_t* crit;  // [BH][Nb][kc]
+  const float* lse;     // [BH][Npad]
+  const float* Drow;    // [BH][Npad]
+  const float* alpha;
+  float* dQs;           // [BH][Npad][128]
+  int* status;
+  int H, N, Npad, Nb, kc;
+  float scale, scale_log2;
+};
+cudaError_t launch_bwd_q_tc(const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                            const __nv_bfloat16* dO, const QTcArgs& a, int BH, cudaStream_t s);
+cudaError_t launch_bwd_kv_tc(const __nv_bfloat16* Q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                             const __nv_bfloat16* dO, const KvTcArgs& a, int BH, cudaStream_t s);
 
 // ---- device helpers ----
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }

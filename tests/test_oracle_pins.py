@@ -434,6 +434,93 @@ def test_quantized_branch_exact_when_inputs_sit_on_the_grids():
     np.testing.assert_allclose(r["O_sq"], r["O_s"] * factor[:, None], rtol=1e-10, atol=1e-12)
 
 
+def test_int8_block_quantisation_ties_go_to_even():
+    # block absmax 127 makes the scale exactly 1, so x / s = x and the codes are
+    # rint(x): halves go to the even neighbour (round-half-away would give
+    # 3, 4, -3, 1, -1, 2 here instead of 2, 4, -2, 0, 0, 2)
+    x = np.zeros((64, 8), dtype=np.float32)
+    x[0, 0] = 127.0
+    x[1, :6] = [2.5, 3.5, -2.5, 0.5, -0.5, 1.5]
+    codes, s = O.quantize_int8_blocks(x, 64)
+    assert s[0] == np.float32(1.0)
+    assert list(codes[1, :6]) == [2, 4, -2, 0, 0, 2]
+    assert codes[0, 0] == 127
+
+
+def test_quantized_branch_folds_each_blocks_v_scale_into_p():
+    # As the grid test above, but the two key blocks' V scales differ by a
+    # factor that is not a power of two (s_v = 1 and 0.75: block 1 holds 0.75
+    # times e4m3 grid values, absmax 336), so the fold r_j = s_v,j / max s_v is
+    # exercised: P of a row whose critical block is j enters as
+    # e4m3(256 r_j c), and O^s_q = O^s e4m3(256 r_j c) / (256 r_j c). A fold
+    # inverted (1 / r_j) or left out (r_j = 1) changes at least one row.
+    rng = np.random.default_rng(77)
+    d, N = 8, 128
+    q = rng.integers(-20, 21, size=(N, d)).astype(np.float32)
+    q[0, 0] = 127
+    q[64, 3] = -127
+    k = np.zeros((N, d), dtype=np.float32)
+    k[:64] = [127, 3, 0, 0, 0, 0, 0, 0]
+    k[64:] = [-127, 5, 1, 0, 0, 0, 0, 0]
+    grid = e4m3_grid()
+    g = rng.choice(grid[grid <= 448], size=(N, d)) * rng.choice([-1, 1], size=(N, d))
+    g[0, 0], g[64, 1] = 448.0, -448.0
+    v = g.copy()
+    v[64:] *= 0.75  # exact in float32: grid values have at most 4 significant bits
+    v = v.astype(np.float32)
+    r = O.forward_head(bits(q), bits(k), bits(v), N, variant="sla2", k_crit=1, k_neg=0, alpha_h=1.0,
+                       quantized=True)
+    _, sv = O.quantize_e4m3_blocks(O.bf16_to_f32(bits(v)), N)
+    assert list(sv) == [1.0, 0.75]
+    crit_block = np.argmax(r["Mc"] == 1, axis=1)
+    assert set(crit_block.tolist()) == {0, 1}  # both folds are used
+    s = np.array([q[i].astype(np.float64) @ k[64 * crit_block[i // 64]] for i in range(N)])
+    x = s / math.sqrt(d) / math.log(2.0)
+    c = 2.0 ** (x - np.ceil(x))
+    rj = np.array([1.0, 0.75])[crit_block[np.arange(N) // 64]]
+
+    def factor(rr):
+        return O.e4m3_round(256.0 * rr * c) / (256.0 * rr * c)
+
+    np.testing.assert_allclose(r["O_sq"], r["O_s"] * factor(rj)[:, None], rtol=1e-10, atol=1e-12)
+    assert np.any(factor(1.0 / rj) != factor(rj)) and np.any(factor(np.ones(N)) != factor(rj))
+
+
+def test_e4m3_p_and_v_alone_exceed_the_low_bit_tolerance_on_the_14b_shape():
+    # A finding about the low-bit scheme itself, not a check of the kernel.
+    # With the scores computed exactly (no INT8 Q or K at all), e4m3 P (the
+    # scheme's power-of-two row scale and V-scale fold) and e4m3 V alone move
+    # the sparse branch by more than the 5e-2 max-abs tolerance stated for the
+    # INT8 / FP8 branch on this workload's peaked rows: three mantissa bits
+    # carry up to 2^-4 relative error per element, and a row dominated by a
+    # few keys passes that error straight to its output. O = alpha O^s +
+    # (1 - alpha) O^l, so O moves by alpha times as much.
+    w = W.WORKLOADS["sla2_q_wan14b_b1h40n75600d128_s97"]
+    inp = W.make_inputs(w, heads=[(0, 5)])
+    q32, k32, v32 = (O.bf16_to_f32(x[0, 0]) for x in (inp.q, inp.k, inp.v))
+    N = w.N
+    m = O.mask_f32_spec(q32, k32, N, w.k_crit, 0, O.bf16_to_f32(inp.proj_q), O.bf16_to_f32(inp.proj_k))
+    vq, sv = O.quantize_e4m3_blocks(v32, N)
+    q, k, v = (x.astype(np.float64) for x in (q32, k32, v32))
+    scale = 1.0 / math.sqrt(w.d)
+    errs, refs = [], []
+    for i in range(0, w.Nb, 30):  # 40 of the 1182 query blocks
+        r0, r1 = i * 64, min(N, (i + 1) * 64)
+        keys = O._block_tokens(np.nonzero(m["Mc"][i] == 1)[0], N)
+        x = (q[r0:r1] @ k[keys].T) * scale * O.LOG2E
+        p = np.exp2(x - np.ceil(x.max(axis=1, keepdims=True)))
+        exact = (p @ v[keys]) / p.sum(axis=1, keepdims=True)
+        rj = (sv[keys // 64] / np.float32(sv.max())).astype(np.float64)
+        pq = O.e4m3_round(p * rj[None, :] * 256.0)
+        low = (pq @ vq[keys]) * (float(sv.max()) / 256.0) / p.sum(axis=1, keepdims=True)
+        errs.append(low - exact)
+        refs.append(exact)
+    e, ref = np.concatenate(errs), np.concatenate(refs)
+    alpha = float(inp.alpha[5])
+    assert alpha * np.abs(e).max() > 5e-2
+    assert np.linalg.norm(e) / np.linalg.norm(ref) > 3e-2
+
+
 def test_quantized_sparse_branch_error_is_quantisation_sized():
     # Diagnostic scale only: on the tiny workload (128 critical keys per row)
     # the low-bit branch stays within a few percent of the exact branch.

@@ -10,10 +10,13 @@ combined with the float64 linear branch. The kernel's P codes are the
 emulation's shifted by a power of two (integer row max), except where the fp32
 exponent and ex2.approx put a P value on the other side of an e4m3 rounding
 midpoint than the float64 one (a rare event per element, frequent over a
-full-size head): that code moves by one e4m3 step. Small cases stay within the bf16 output contract; the full-size
-case is held to the low-bit output tolerance (5e-2 max-abs, 3e-2 rel-L2). The
-distance to the exact (unquantised) output is the scheme's own error; it is
-checked against the diagnostic bound the oracle's own pins use.
+full-size head): that code moves by one e4m3 step. Small cases stay within the
+bf16 output contract; the full-size case is held to the low-bit output
+tolerance (5e-2 max-abs, 3e-2 rel-L2) against that emulation. Against the
+exact (unquantised) output the scheme's own error is checked against a
+diagnostic bound (rel-L2 < 0.1); the stated low-bit tolerance against the
+unquantised output is a strict xfail: the scheme misses it on this workload
+whatever the kernel does (see the oracle pin on e4m3 P and V).
 """
 
 import numpy as np
@@ -110,13 +113,23 @@ def test_quantized_phi_elu1(cuda_lib, record_property):
     check_outputs(inp, res, [0, 1], record_property)
 
 
-@pytest.mark.slow
-def test_quantized_full_size_wan14b(cuda_lib, record_property):
-    """The 40-head, 75,600-token SLA2 workload at 97 % sparsity: codes and
-    scales of every head, the mask of eight heads, the output of two."""
+@pytest.fixture(scope="module")
+def wan14b(cuda_lib):
+    """One run of the 40-head, 75,600-token SLA2 workload at 97 % sparsity and
+    the oracle (with the emulated low-bit branch) of heads 5 and 31."""
     w = W.WORKLOADS["sla2_q_wan14b_b1h40n75600d128_s97"]
     inp = W.make_inputs(w)
     res = run_library(cuda_lib, inp)
+    refs = {idx: oracle_head(inp, idx, quantized=True) for idx in (5, 31)}
+    return inp, res, refs
+
+
+@pytest.mark.slow
+def test_quantized_full_size_wan14b(cuda_lib, wan14b, record_property):
+    """Codes and scales of every head, the mask of eight heads, the output of
+    two against the emulation of the same low-bit scheme."""
+    inp, res, refs = wan14b
+    w = inp.w
     assert res["status"] == 0
     check_codes(cuda_lib, inp, res, range(w.B * w.H))
     for idx in (0, 7, 13, 19, 22, 28, 33, 39):
@@ -124,3 +137,25 @@ def test_quantized_full_size_wan14b(cuda_lib, record_property):
         b, h = inp.heads[idx]
         np.testing.assert_array_equal(res["Mc"][b, h], m["Mc"], err_msg=f"mask head {idx}")
     check_outputs(inp, res, [5, 31], record_property, Q_MAX_ABS, Q_REL_L2)
+
+
+@pytest.mark.slow
+@pytest.mark.xfail(strict=True, reason=(
+    "the low-bit scheme itself misses 5e-2 / 3e-2 against the unquantised output on this "
+    "workload: e4m3 P and V alone, with exact scores, already exceed it (oracle pin "
+    "test_e4m3_p_and_v_alone_exceed_the_low_bit_tolerance_on_the_14b_shape); measured "
+    "about 0.24 max-abs and 5 % rel-L2 for the whole scheme"))
+def test_quantized_full_size_wan14b_meets_low_bit_tolerance_vs_unquantised_oracle(wan14b, record_property):
+    """The stated INT8 / FP8 tolerance (max-abs 5e-2, rel-L2 3e-2) against the
+    unquantised float64 output. Strict xfail: if a scheme ever meets it, this
+    test reports XPASS as a failure so the expectation gets updated."""
+    inp, res, refs = wan14b
+    N = inp.w.N
+    worst = (0.0, 0.0)
+    for idx, r in refs.items():
+        b, h = inp.heads[idx]
+        ma, rl = errors(res["O"][b, h][:N], r["O"])
+        worst = (max(worst[0], ma), max(worst[1], rl))
+    record_property("max_abs_vs_unquantised", worst[0])
+    record_property("rel_l2_vs_unquantised", worst[1])
+    assert worst[0] <= Q_MAX_ABS and worst[1] <= Q_REL_L2, worst
