@@ -44,7 +44,7 @@ LOWBIT_OVER_BF16 = 2.0
 # this build's attention kernel (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by workload; a workload without a capture of the current kernel gets
 # null
-ATTN_TRAFFIC = {"sla_wan13b_b1h12n32768d128_s95": 421516288 + 91559424}
+ATTN_TRAFFIC = {}
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "ms/forward and dense-equiv TFLOPS at 95-97% sparsity; tensor-pipe % of B200 peak"
 UNIT = "TFLOPS (dense-equivalent)"
@@ -240,14 +240,36 @@ def lowbit_peaks(bf16_burst):
     return out
 
 
+def stream_chunks(w):
+    """Chunks per head of the K / V pass (one partial H and Z each): the
+    streaming path (bf16, d = 128) sizes them for about 296 CTAs, the general
+    path takes 512 tokens per chunk."""
+    if w.precision == "bf16" and w.d == 128:
+        per_head = max(1, min(w.Nb, 296 // max(1, w.B * w.H)))
+        cb = -(-w.Nb // per_head)
+    else:
+        cb = 8
+    return -(-w.Nb // cb)
+
+
 def stage_bytes(w):
-    """Bytes each memory-bound stage moves (reads + writes) in this design."""
+    """Bytes each memory-bound stage moves (reads + writes) in this design.
+    pool: Q read, pooled vectors written, phi(Q) written when the linear
+    branch takes it precomputed; the general path (d = 64 or the quantised
+    branch) reads K here too. phik_hz: K and V read, phi(K), z_j and the
+    chunks' partial H, Z written; the streaming path also writes the pooled K."""
     BH, N, Np, Nb, d = w.B * w.H, w.N, w.N_pad, w.Nb, w.d
-    nchunk = (Np + 511) // 512
-    return {
-        "pool": BH * (2 * N * d * 2 + 2 * Nb * d * 4),
-        "phik_hz": BH * (2 * N * d * 2 + Np * d * 2 + Nb * d * 4 + nchunk * d * d * 4),
-    }
+    stream = w.precision == "bf16" and w.d == 128
+    linear = w.k_crit + w.k_neg < Nb
+    pre = linear and (w.precision != "bf16" or w.k_neg * 1260 < (w.k_crit + w.k_neg) * 350 + 8000)
+    nchunk = stream_chunks(w)
+    pool = N * d * 2 + Nb * d * 4 + (N * d * 2 if pre else 0)
+    kv = 2 * N * d * 2 + Np * d * 2 + Nb * d * 4 + nchunk * (d * d + d) * 4
+    if stream:
+        kv += Nb * d * 4
+    else:
+        pool += N * d * 2 + Nb * d * 4
+    return {"pool": BH * pool, "phik_hz": BH * kv}
 
 
 # ---------------------------------------------------------------------------

@@ -299,9 +299,12 @@ sla_status sla_forward_noalloc(const void* Q, const void* K, const void* V, void
                                const sla_params* p, void* stream);
 
 /* Stage timing, a profiling aid (no counterpart on the pages). Stages of
- * sla_forward, in order: 0 pooling (+ router), 1 pooled scores, 2 classification,
- * 3 phi(K) / z_j / partial H, 4 H_tot / Z_tot reduction, 5 attention (sparse +
- * linear + combine). */
+ * sla_forward, in order: 0 the Q-side pass (pooling of Q, + router; phi(Q) when
+ * the linear branch takes it precomputed; at d = 64 or with the quantised
+ * branch also the pooling of K and the INT8 codes), 1 the K / V pass (at d = 128
+ * in bf16 also the pooling of K; phi(K), z_j, partial H and Z), 2 pooled
+ * scores, 3 classification, 4 H_tot / Z_tot reduction (and Z_i), 5 attention
+ * (sparse + linear + combine). */
 #define SLA_NUM_STAGES 6
 
 /* max_calls > 0: create CUDA events (on the current device) for up to max_calls

@@ -42,7 +42,7 @@ EXPORTS = ("sla_abi_version", "sla_status_string", "sla_validate", "sla_workspac
            "sla_backward", "sla_check_wait_timeout")
 NOALLOC_WORKSPACE_BYTES = 32 << 20
 NUM_STAGES = 6
-STAGES = ("pool", "scores", "classify", "phik_hz", "hz_reduce", "attention")
+STAGES = ("pool", "phik_hz", "scores", "classify", "hz_reduce", "attention")
 
 
 class Params(ctypes.Structure):

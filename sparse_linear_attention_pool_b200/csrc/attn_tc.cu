@@ -55,6 +55,7 @@ using namespace tc;
 
 struct TcMaps {
   CUtensorMap q, k, v, phik, w, phiq, o;
+  CUtensorMap ht;  // H_tot in bf16, [BH][d][d] (d = 128)
   CUtensorMap qc, kc, vc;  // INT8 Q, K and e4m3 V codes (quantised sparse branch)
 };
 
@@ -84,6 +85,8 @@ struct TcCfg {
   static constexpr int cO = 128;               // O: D columns
   static constexpr int cG = 128 + D;           // G_A (D=128: G_B at cG + 128; D=64: M=64 halves)
   static constexpr int cNumA = 0;              // num of block A (over S, after the loop)
+  // d = 128: phi(Q) H_tot over S, phi(Q) (-G_A) over G_A, phi(Q) (-G_B) over G_B
+  static constexpr int cT = 0, cNegA = cG, cNegB = cG + 128;
   static constexpr int cNumB = D == 128 ? cG : 64;        // num of block B (over G_A / S)
   static constexpr int cY = D == 128 ? cG + 128 : cG;     // Y = O^l W (over G_B / G)
   static constexpr uint32_t kTmemCols = D == 128 ? 512 : 256;
@@ -94,7 +97,7 @@ enum Bar {
   bKFull0, bKFull1, bKFull2, bKEmpty0, bKEmpty1, bKEmpty2, bKDone0, bKDone1, bKDone2,
   bVFull0, bVFull1, bVEmpty0, bVEmpty1,
   bSFull, bSFree, bPFull, bPvDone,
-  bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, bQFree, bPhiQFull, kNumBars
+  bTailDone, bHiFull, bNumFull, bWFull, bOlFull, bYFull, bDrain, bQFree, bPhiQFull, bHtFull, kNumBars
 };
 
 // QNT: the sparse branch on the quantised forms (SLA2 article, quantisation
@@ -145,6 +148,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   // negligible blocks only. The quantised branch keeps V as e4m3 codes in
   // phase 1 and so takes every excluded block in phase 2.
   constexpr bool kMergeCapable = !QNT && MODE != kModeDense && D == 128;
+  // d = 128: the linear numerator is phi(Q) H_tot (H_tot loaded as a bf16 tile)
+  // plus phi(Q) (-G_X); d = 64 forms H_X = H_tot - G_X from the fp32 H_tot
+  constexpr bool kHtTile = D == 128 && MODE != kModeDense;
   const bool merge = kMergeCapable && has_marg;
   // phi(Q) and Z_i precomputed (loaded) rather than formed in the epilogue
   const bool pre = has_marg && a.phiq != nullptr;
@@ -222,6 +228,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     mbar_init(bar(bDrain), 1);
     mbar_init(bar(bQFree), 1);
     mbar_init(bar(bPhiQFull), 1);
+    mbar_init(bar(bHtFull), 1);
     fence_barrier_init();
   }
   if (warp == 5) tmem_alloc(smem_u32(&tmem_base_sh), C::kTmemCols);
@@ -433,6 +440,21 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       }
     }
     if (pre && !merge && !stop) load_phiq();
+    // d = 128: H_tot (bf16) into the V slot the next fill would take, once the
+    // products that read that slot's last V have completed
+    bool ht_issued = false;
+    if (kHtTile && has_marg && !stop) {
+      const int sv = nTot % C::kNV;
+      if (pwait(bVEmpty0 + sv, ((nTot / C::kNV) & 1) ^ 1)) {
+        if (lane == 0) {
+          mbar_expect_tx(bar(bHtFull), C::kMat);
+          tma_load_3d(sV + sv * C::kPair, &maps.ht, bar(bHtFull), 0, 0, bh);
+          tma_load_3d(sV + sv * C::kPair + D * 128, &maps.ht, bar(bHtFull), 64, 0, bh);
+        }
+        ht_issued = true;
+      }
+      __syncwarp();
+    }
     bool w_issued = false;
     if (use_y && pwait(bTailDone, 0)) {  // W reuses the rings once every loop product has completed
       if (lane == 0) {
@@ -449,6 +471,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       for (int st = 0; st < C::kNV; ++st)
         if ((vany >> st) & 1u) wait_drain(bVFull0 + st, ((vpar >> st) & 1u) ^ 1u);
       if (phiq_issued) wait_drain(bPhiQFull, 0);
+      if (ht_issued) wait_drain(bHtFull, 0);
       if (w_issued) wait_drain(bWFull, 0);
     }
     __syncwarp();
@@ -567,14 +590,28 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       mma_commit(bar(bTailDone));
       if (has_marg) {
         wait_w(bHiFull, 0);
+        if constexpr (kHtTile) wait_w(bHtFull, 0);
         tc_fence_after();
-        // [phi(Q_A); phi(Q_B)] H_A and [phi(Q_A); phi(Q_B)] H_B: the A rows of
-        // the first and the B rows of the second are kept
+        if constexpr (kHtTile) {
+          // T = [phi(Q_A); phi(Q_B)] H_tot (both blocks' rows kept) and
+          // [phi(Q_A); phi(Q_B)] (-G_X) for X = A, B (the rows of block X kept)
+          const uint32_t sHt = sV + (nTot % C::kNV) * C::kPair;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * C::kSubS + (k & 3) * 32;
-          mma_bf16(tb + C::cNumA, sdesc(sQ + off, 16, 1024), sdesc(sHA + k * 2048, D * 128, 1024), idN, k > 0);
-          mma_bf16(tb + C::cNumB, sdesc(sQ + off, 16, 1024), sdesc(sHB + k * 2048, D * 128, 1024), idN, k > 0);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * C::kSubS + (k & 3) * 32;
+            mma_bf16(tb + C::cT, sdesc(sQ + off, 16, 1024), sdesc(sHt + k * 2048, D * 128, 1024), idN, k > 0);
+            mma_bf16(tb + C::cNegA, sdesc(sQ + off, 16, 1024), sdesc(sHA + k * 2048, D * 128, 1024), idN, k > 0);
+            mma_bf16(tb + C::cNegB, sdesc(sQ + off, 16, 1024), sdesc(sHB + k * 2048, D * 128, 1024), idN, k > 0);
+          }
+        } else {
+          // [phi(Q_A); phi(Q_B)] H_A and [phi(Q_A); phi(Q_B)] H_B: the A rows of
+          // the first and the B rows of the second are kept
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * C::kSubS + (k & 3) * 32;
+            mma_bf16(tb + C::cNumA, sdesc(sQ + off, 16, 1024), sdesc(sHA + k * 2048, D * 128, 1024), idN, k > 0);
+            mma_bf16(tb + C::cNumB, sdesc(sQ + off, 16, 1024), sdesc(sHB + k * 2048, D * 128, 1024), idN, k > 0);
+          }
         }
         mma_commit(bar(bNumFull));
       }
@@ -621,6 +658,17 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     const int jlast = dense ? Nb - 1 : checked((isB ? critB : critA)[nA - 1]);
     const bool mask_last = jlast * 64 + 64 > N;
     float m = -INFINITY, l = 0.0f;
+    // precomputed Z_i of blocks A and B, read now so that the epilogue does not wait for it
+    float zpre[2] = {0.0f, 0.0f};
+    if (pre) {
+      const float* zia = a.zi + (size_t(bh) * Nb + iA) * D;
+      const float* zib = a.zi + (size_t(bh) * Nb + iB) * D;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = tid + 128 * k;
+        if (e < 2 * D) zpre[k] = (e < D ? zia : zib)[e % D];
+      }
+    }
     // quantised branch: the row's INT8 scale and the head's largest V scale
     float q_scale = 1.0f, sv_max = 1.0f;
     if constexpr (QNT) {
@@ -757,14 +805,13 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 
     float den = 1.0f;
     if (pre) {
-      // Z_i of blocks A and B (precomputed), then den = phi(Q_i) . Z_i from the
-      // phi(Q) tile the producer loads over Q once the last S product is done
-      const float* zia = a.zi + (size_t(bh) * Nb + iA) * D;
-      const float* zib = a.zi + (size_t(bh) * Nb + iB) * D;
+      // Z_i of blocks A and B (precomputed, loaded before the loop), then
+      // den = phi(Q_i) . Z_i from the phi(Q) tile the producer loads over Q
+      // once the last S product is done
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int e = tid + 128 * k;
-        if (e < 2 * D) zs[e / D][e % D] = (e < D ? zia : zib)[e % D];
+        if (e < 2 * D) zs[e / D][e % D] = zpre[k];
       }
       named_bar(1, 128);  // zs complete
       wait_w(bPhiQFull, 0);
@@ -855,7 +902,37 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         *qchunk(c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
-    if (has_marg) {
+    if (has_marg && kHtTile) {
+      // -G_A, -G_B -> bf16, MN-major tiles [D rows c][D cols e] (G row c =
+      // TMEM lane c); the numerator is then phi(Q) H_tot + phi(Q) (-G_X)
+      wait_w(bTailDone, 0);
+      tc_fence_after();
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        float g[2][32];
+        tmem_ld32(tq + C::cG + ch * 32, g[0]);
+        tmem_ld32(tq + C::cG + 128 + ch * 32, g[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          unsigned char* Hbase = smem + (X ? C::oHB : C::oHA);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const int e0 = ch * 32 + q8 * 8;
+            const float* gx = g[X] + q8 * 8;
+            const uint4 v = make_uint4(pack_bf16(-gx[0], -gx[1]), pack_bf16(-gx[2], -gx[3]),
+                                       pack_bf16(-gx[4], -gx[5]), pack_bf16(-gx[6], -gx[7]));
+            *reinterpret_cast<uint4*>(Hbase + (e0 >> 6) * (D * 128) + sw128_chunk(tid, (e0 & 63) >> 3)) = v;
+          }
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      named_bar(1, 128);
+      if (tid == 0) mbar_arrive(bar(bHiFull));
+      wait_w(bNumFull, 0);
+      tc_fence_after();
+    } else if (has_marg) {
       // H_i = H_tot - G_i -> bf16, MN-major tile [D rows c][D cols e]
       // D=128: G rows c = TMEM lanes (M = 128), G_A and G_B in separate columns;
       // D=64:  G_A rows in lanes 0-15 of each quarter, G_B in lanes 16-31.
@@ -922,6 +999,20 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       a.save_lse[sidx] = (m + log2f(l)) * 0.69314718055994531f;
       a.save_den[sidx] = has_marg ? den : 0.0f;
     }
+    // this row's linear numerator, columns 32 ch .. 32 ch + 31
+    auto load_num = [&](int ch, float (&x)[32]) {
+      if constexpr (kHtTile) {
+        float ng[32];
+        tmem_ld32(tq + C::cT + ch * 32, x);
+        tmem_ld32(tq + (isB ? C::cNegB : C::cNegA) + ch * 32, ng);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] += ng[i];
+      } else {
+        tmem_ld32(tq + (isB ? C::cNumB : C::cNumA) + ch * 32, x);
+        tmem_wait_ld();
+      }
+    };
     // O is staged as a bf16 pair tile in the P region (free after the last PV)
     // and written by TMA; the tensor map's row extent N drops the pad rows
     unsigned char* Ot = smem + C::oP;
@@ -931,8 +1022,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
         float nm[32];
-        tmem_ld32(tq + (isB ? C::cNumB : C::cNumA) + ch * 32, nm);
-        tmem_wait_ld();
+        load_num(ch, nm);
         if (srow) save_row(a.save_ol, ch, nm, inv_den);
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
@@ -954,9 +1044,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 #pragma unroll 1
     for (int ch = 0; ch < D / 32; ++ch) {
       float o[32], x[32];
-      tmem_ld32(tq + C::cO + ch * 32, o);
       if (use_y) tmem_ld32(tq + C::cY + ch * 32, x);
-      else if (has_marg) tmem_ld32(tq + (isB ? C::cNumB : C::cNumA) + ch * 32, x);
+      else if (has_marg) load_num(ch, x);
+      tmem_ld32(tq + C::cO + ch * 32, o);
       tmem_wait_ld();
       float out[32];
 #pragma unroll
@@ -1007,35 +1097,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
 // ---------------------------------------------------------------------------
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [BH][rows_alloc][D] bf16 viewed as 3D (D, rows, BH); rows >= rows_valid read as zero.
-bool map_rows(CUtensorMap* m, const void* base, int D, int rows_valid, int rows_alloc, int BH) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(rows_valid), cuuint64_t(BH)};
-  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(rows_alloc) * D * 2};
-  cuuint32_t box[3] = {64, 64, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
+using tc::EncodeTiledFn;
+using tc::encode_fn;
+using tc::map_rows;
 
 // [D][D] bf16 (row = input dim), boxes of 64 columns x D rows.
 bool map_square(CUtensorMap* m, const void* base, int D) {
@@ -1046,6 +1110,19 @@ bool map_square(CUtensorMap* m, const void* base, int D) {
   cuuint32_t box[2] = {64, cuuint32_t(D)};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [BH][D][D] bf16 (a matrix per head, row = input dim), boxes of 64 columns x D rows.
+bool map_square_heads(CUtensorMap* m, const void* base, int D, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(D), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(D) * D * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(D), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1086,6 +1163,8 @@ cudaError_t launch_attention(const AttnArgs& a, int BH, int d, int mode, cudaStr
   if (ok && a.phiq) ok = map_rows(&maps.phiq, a.phiq, d, a.N, Npad, BH);
   if (ok) ok = map_rows(&maps.o, a.O, d, a.N, Npad, BH);
   if (ok && a.w_proj) ok = map_square(&maps.w, a.w_proj, d);
+  if (ok && d == 128 && mode != kModeDense)  // the d = 128 epilogue reads H_tot as a bf16 tile
+    ok = a.htot16 != nullptr && map_square_heads(&maps.ht, a.htot16, d, BH);
   const bool quant = a.qcode != nullptr;
   // the quantised branch's Q tiles hold INT8 codes: its phi(Q) must come precomputed
   if (quant && a.kc + a.kn < a.Nb && a.phiq == nullptr) return cudaErrorInvalidValue;

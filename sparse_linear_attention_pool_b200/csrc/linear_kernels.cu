@@ -263,14 +263,18 @@ __device__ __forceinline__ float strided_sum(const float* __restrict__ src, int 
 __global__ void __launch_bounds__(256) hz_reduce_kernel(const float* __restrict__ zpart,
                                                         const float* __restrict__ hpart,
                                                         float* __restrict__ htot32,
+                                                        __nv_bfloat16* __restrict__ htot16,
                                                         float* __restrict__ ztot, int nchunk, int d) {
   const int bh = blockIdx.y;
   const size_t dd = size_t(d) * d;
   const int nh = int((dd + 255) / 256);
   if (int(blockIdx.x) < nh) {
     const int e = blockIdx.x * 256 + threadIdx.x;
-    if (e < int(dd))
-      htot32[size_t(bh) * dd + e] = strided_sum(hpart + size_t(bh) * nchunk * dd + e, nchunk, dd);
+    if (e < int(dd)) {
+      const float v = strided_sum(hpart + size_t(bh) * nchunk * dd + e, nchunk, dd);
+      htot32[size_t(bh) * dd + e] = v;
+      htot16[size_t(bh) * dd + e] = __float2bfloat16_rn(v);
+    }
   } else if (threadIdx.x < d) {
     ztot[size_t(bh) * d + threadIdx.x] =
         strided_sum(zpart + size_t(bh) * nchunk * d + threadIdx.x, nchunk, size_t(d));
@@ -278,9 +282,9 @@ __global__ void __launch_bounds__(256) hz_reduce_kernel(const float* __restrict_
 }
 
 cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* hpart, float* htot32,
-                             float* ztot, cudaStream_t s) {
+                             __nv_bfloat16* htot16, float* ztot, cudaStream_t s) {
   dim3 grid((L.d * L.d + 255) / 256 + 1, L.BH);
-  hz_reduce_kernel<<<grid, 256, 0, s>>>(zpart, hpart, htot32, ztot, L.nchunk, L.d);
+  hz_reduce_kernel<<<grid, 256, 0, s>>>(zpart, hpart, htot32, htot16, ztot, L.nchunk, L.d);
   return cudaGetLastError();
 }
 

@@ -210,7 +210,8 @@ cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bflo
 // ---------------------------------------------------------------------------
 // CTA: 16 x 16 threads, a 64 x 128 tile of S; thread (tx, ty) owns rows
 // ty + 16a (a < 4) and columns tx + 16b (b < 8). k runs ascending across
-// 32-wide chunks.
+// 32-wide chunks; the next chunk's values are loaded into registers while the
+// current one is multiplied, so the global loads overlap the arithmetic.
 __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ qbar,
                                                      const float* __restrict__ kbar,
                                                      float* __restrict__ S, int Nb, int d) {
@@ -225,18 +226,28 @@ __global__ void __launch_bounds__(256) scores_kernel(const float* __restrict__ q
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
-  for (int k0 = 0; k0 < d; k0 += 32) {
+  // this thread's share of a chunk: rows it * 8 + tid / 32, column tid % 32
+  float qn[8], kn[16];
+  auto fetch = [&](int k0) {
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
       const int r = it * 8 + tid / 32, c = tid % 32;
-      Qs[r][c] = (i0 + r < Nb) ? qb[size_t(i0 + r) * d + k0 + c] : 0.0f;
+      qn[it] = (i0 + r < Nb) ? qb[size_t(i0 + r) * d + k0 + c] : 0.0f;
     }
 #pragma unroll
     for (int it = 0; it < 16; ++it) {
       const int r = it * 8 + tid / 32, c = tid % 32;
-      Ks[r][c] = (j0 + r < Nb) ? kb[size_t(j0 + r) * d + k0 + c] : 0.0f;
+      kn[it] = (j0 + r < Nb) ? kb[size_t(j0 + r) * d + k0 + c] : 0.0f;
     }
+  };
+  fetch(0);
+  for (int k0 = 0; k0 < d; k0 += 32) {
+#pragma unroll
+    for (int it = 0; it < 8; ++it) Qs[it * 8 + tid / 32][tid % 32] = qn[it];
+#pragma unroll
+    for (int it = 0; it < 16; ++it) Ks[it * 8 + tid / 32][tid % 32] = kn[it];
     __syncthreads();
+    if (k0 + 32 < d) fetch(k0 + 32);
 #pragma unroll 4
     for (int kk = 0; kk < 32; ++kk) {
       float qv[4], kv[8];

@@ -104,6 +104,7 @@ sla_status run_forward(const void* Q, const void* K, const void* V, void* O, con
   float* hpart = reinterpret_cast<float*>(ws + L.hpart);
   float* zpart = reinterpret_cast<float*>(ws + L.zpart);
   float* htot32 = reinterpret_cast<float*>(ws + L.htot32);
+  __nv_bfloat16* htot16 = reinterpret_cast<__nv_bfloat16*>(ws + L.htot16);
   float* ztot = reinterpret_cast<float*>(ws + L.ztot);
   __nv_bfloat16* phiq = L.pre ? reinterpret_cast<__nv_bfloat16*>(ws + L.phiq) : nullptr;
   float* zi = L.pre ? reinterpret_cast<float*>(ws + L.zi) : nullptr;
@@ -120,21 +121,33 @@ sla_status run_forward(const void* Q, const void* K, const void* V, void* O, con
   auto mark = [&](int k) {
     if (call >= 0) cudaEventRecord(stage_event(call, k), s);
   };
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  const __nv_bfloat16* proj_q = sla2 ? bf(p->proj_q) : nullptr;
+  const __nv_bfloat16* proj_k = sla2 ? bf(p->proj_k) : nullptr;
   cudaError_t e = cudaMemsetAsync(ws + L.status, 0, 256, s);
+  // stages: 0 Q side (pooling; phi(Q) when precomputed; the general path pools
+  // K here too), 1 K / V side (phi(K), z_j, partial H and Z), 2 scores,
+  // 3 classification, 4 H_tot / Z_tot (and Z_i), 5 attention
   mark(0);
-  if (e == cudaSuccess)
-    e = launch_pool(L, bf(Q), bf(K), sla2 ? bf(p->proj_q) : nullptr, sla2 ? bf(p->proj_k) : nullptr,
-                    qbar, kbar, qcode, kcode, qscale, kscale, phiq, elu1, s);
-  mark(1);
-  if (e == cudaSuccess) e = launch_scores(L, qbar, kbar, scores, s);
+  if (L.stream) {
+    if (e == cudaSuccess) e = launch_q_stream(L, bf(Q), proj_q, qbar, phiq, elu1, status, s);
+    mark(1);
+    if (e == cudaSuccess)
+      e = launch_kv_stream(L, bf(K), bf(V), proj_k, kbar, phik, zblk, hpart, zpart, elu1, status, s);
+  } else {
+    if (e == cudaSuccess)
+      e = launch_pool(L, bf(Q), bf(K), proj_q, proj_k, qbar, kbar, qcode, kcode, qscale, kscale, phiq, elu1, s);
+    mark(1);
+    if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, zpart, vcode, vscale, elu1, s);
+  }
   mark(2);
-  if (e == cudaSuccess) e = launch_classify(L, scores, mc, crit, neg, s);
+  if (e == cudaSuccess) e = launch_scores(L, qbar, kbar, scores, s);
   mark(3);
-  if (e == cudaSuccess) e = launch_phik_hz(L, bf(K), bf(V), phik, zblk, hpart, zpart, vcode, vscale, elu1, s);
+  if (e == cudaSuccess) e = launch_classify(L, scores, mc, crit, neg, s);
   mark(4);
-  if (e == cudaSuccess) e = launch_hz_reduce(L, zpart, hpart, htot32, ztot, s);
+  if (e == cudaSuccess) e = launch_hz_reduce(L, zpart, hpart, htot32, htot16, ztot, s);
   if (e == cudaSuccess && L.pre)
-    e = launch_zi(L, crit, neg, zblk, ztot, zi, reinterpret_cast<int*>(ws + L.status), s);
+    e = launch_zi(L, crit, neg, zblk, ztot, zi, status, s);
   mark(5);
   if (e == cudaSuccess) {
     AttnArgs a{};
@@ -146,6 +159,7 @@ sla_status run_forward(const void* Q, const void* K, const void* V, void* O, con
     a.crit = crit;
     a.neg = neg;
     a.htot32 = htot32;
+    a.htot16 = htot16;
     a.phiq = phiq;
     a.zi = zi;
     a.ztot = ztot;

@@ -2,6 +2,8 @@
 // workspace layout, launcher prototypes and small device helpers.
 #pragma once
 
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -21,17 +23,25 @@ enum DeviceStatus : int { kDevOk = 0, kDevTimeout = 1, kDevBadIndex = 2 };
 // device (looked up once per device; defined in noalloc.cu).
 sla_status noalloc_workspace_address(void** out);
 
-// Tokens per CTA in the phi(K) / h / z pass (8 blocks).
+// Tokens per CTA in the phi(K) / h / z pass of the general path (8 blocks).
 constexpr int kHzChunk = 512;
+// The streaming passes (bf16, d = 128) split each head into chunks of
+// consecutive blocks so that the grid is about this many CTAs: two per SM of
+// a 148-SM B200, one wave.
+constexpr int kStreamCtas = 296;
 
 // Derived sizes and the byte offsets of every workspace region.
 struct Layout {
-  int B, H, BH, N, Npad, Nb, d, kc, kn, nchunk;
+  int B, H, BH, N, Npad, Nb, d, kc, kn;
+  int nchunk;     // chunks per head of the phi(K) / h / z pass (one partial H, Z each)
+  int stream_cb;  // blocks per chunk
+  bool stream;    // bf16 at d = 128: q_stream / kv_stream kernels (pool, phi and
+                  // the partial sums in two passes over Q and K, V)
   bool quant;  // INT8 / FP8 sparse branch: regions qcode .. vscale are present
   bool linear;  // a marginal block exists (the linear branch is computed)
   bool pre;     // phi(Q) and Z_i are precomputed (regions phiq, zi) instead of
                 // formed inside the attention kernel
-  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, zpart, htot32, ztot, phiq, zi;
+  size_t status, qbar, kbar, scores, mc, crit, neg, phik, zblk, hpart, zpart, htot32, htot16, ztot, phiq, zi;
   size_t qcode, kcode, vcode, qscale, kscale, vscale, total;
 };
 
@@ -46,7 +56,15 @@ inline Layout make_layout(const sla_params& p) {
   L.d = p.d;
   L.kc = p.k_crit;
   L.kn = p.k_neg;
-  L.nchunk = (L.Npad + kHzChunk - 1) / kHzChunk;
+  L.quant = p.precision == SLA_PREC_I8QK_F8PV;
+  L.stream = p.d == 128 && !L.quant;
+  if (L.stream) {
+    const int per_head = std::max(1, std::min(L.Nb, kStreamCtas / std::max(1, L.BH)));
+    L.stream_cb = (L.Nb + per_head - 1) / per_head;
+  } else {
+    L.stream_cb = kHzChunk / kBlock;
+  }
+  L.nchunk = (L.Nb + L.stream_cb - 1) / L.stream_cb;
   const size_t BH = size_t(L.BH), Nb = size_t(L.Nb), d = size_t(L.d);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -66,6 +84,7 @@ inline Layout make_layout(const sla_params& p) {
   L.hpart = take(BH * size_t(L.nchunk) * d * d * 4);
   L.zpart = take(BH * size_t(L.nchunk) * d * 4);
   L.htot32 = take(BH * d * d * 4);
+  L.htot16 = take(BH * d * d * 2);
   L.ztot = take(BH * d * 4);
   L.linear = L.kc + L.kn < L.Nb;
   // The attention kernel forms Z_i (about 350 cycles per excluded block) and
@@ -77,7 +96,6 @@ inline Layout make_layout(const sla_params& p) {
                        size_t(L.kn) * 1260 < size_t(L.kc + L.kn) * 350 + 8000);
   L.phiq = take(L.pre ? BH * size_t(L.Npad) * d * 2 : 0);  // phi(Q) bf16 [BH, Npad, d]
   L.zi = take(L.pre ? BH * Nb * d * 4 : 0);               // Z_i fp32 [BH, Nb, d]
-  L.quant = p.precision == SLA_PREC_I8QK_F8PV;
   const size_t codes = L.quant ? BH * size_t(L.Npad) * d : 0;
   const size_t scales = L.quant ? BH * Nb * 4 : 0;
   L.qcode = take(codes);  // int8 [BH, Npad, d]
@@ -97,12 +115,19 @@ cudaError_t launch_pool(const Layout& L, const __nv_bfloat16* Q, const __nv_bflo
                         __nv_bfloat16* phiq, int phi_elu1, cudaStream_t s);
 cudaError_t launch_scores(const Layout& L, const float* qbar, const float* kbar, float* scores,
                           cudaStream_t s);
+// streaming passes (L.stream): Q side (qbar, phi(Q) when phiq != null) and
+// K / V side (kbar, phi(K), z_j, the chunks' partial H and Z)
+cudaError_t launch_q_stream(const Layout& L, const __nv_bfloat16* Q, const __nv_bfloat16* proj_q, float* qbar,
+                            __nv_bfloat16* phiq, int phi_elu1, int* status, cudaStream_t s);
+cudaError_t launch_kv_stream(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                             const __nv_bfloat16* proj_k, float* kbar, __nv_bfloat16* phik, float* zblk,
+                             float* hpart, float* zpart, int phi_elu1, int* status, cudaStream_t s);
 cudaError_t launch_classify(const Layout& L, const float* scores, int8_t* mc, int32_t* crit,
                             int32_t* neg, cudaStream_t s);
 cudaError_t launch_phik_hz(const Layout& L, const __nv_bfloat16* K, const __nv_bfloat16* V,
                            __nv_bfloat16* phik, float* zblk, float* hpart, float* zpart,
                            uint8_t* vcode, float* vscale, int phi_elu1, cudaStream_t s);
-cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* hpart, float* htot32,
+cudaError_t launch_hz_reduce(const Layout& L, const float* zpart, const float* hpart, float* htot32, __nv_bfloat16* htot16,
                              float* ztot, cudaStream_t s);
 // Z_i = Z_tot - sum of z_j over the excluded blocks of query block i
 cudaError_t launch_zi(const Layout& L, const int32_t* crit, const int32_t* neg, const float* zblk,
@@ -120,6 +145,7 @@ struct AttnArgs {
   const int32_t* crit;         // [BH, Nb, kc]
   const int32_t* neg;          // [BH, Nb, kn]
   const float* htot32;         // [BH, d, d]  H_tot = sum_j phi(K_j)^T V_j
+  const __nv_bfloat16* htot16; // [BH, d, d]  H_tot rounded to bf16 (read at d = 128)
   const __nv_bfloat16* phiq;   // [BH, Npad, d] phi(Q), or null: formed in the kernel
   const float* zi;             // [BH, Nb, d] Z_i, or null: formed in the kernel
   const float* ztot;           // [BH, d] Z_tot (in-kernel Z_i)
