@@ -44,7 +44,8 @@ LOWBIT_OVER_BF16 = 2.0
 # this build's attention kernel (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by workload; a workload without a capture of the current kernel gets
 # null
-ATTN_TRAFFIC = {}
+ATTN_TRAFFIC = {"sla_wan13b_b1h12n32768d128_s95": 417141248 + 91571200,
+                "sla2_b1h12n32768d128_s97": 511963392 + 92794368}
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "ms/forward and dense-equiv TFLOPS at 95-97% sparsity; tensor-pipe % of B200 peak"
 UNIT = "TFLOPS (dense-equivalent)"
@@ -706,7 +707,7 @@ def run_ours(args):
                  "executed_excl_masked_tflops": round(useful_flops(w97) / t97 / 1e12, 2),
                  "executed_excl_masked_frac": round(useful_flops(w97) / t97 / 1e12 / pk97, 4),
                  "issued_tflops": round(executed_flops(w97) / t97 / 1e12, 2),
-                 "peak": pk97, "peak_kind": pk97_kind,
+                 "peak": pk97, "peak_kind": pk97_kind, "traffic": ATTN_TRAFFIC.get(w97.name),
                  "attention_l2_fill": fill97}
         if "dense_baseline" in res:
             entry["speedup_vs_dense"] = round(res["dense_baseline"]["ms"] / ms97, 3)
@@ -830,6 +831,19 @@ def run_backward_only(args):
                       "dense_flash_backward_ms": None if dms is None else round(dms, 4)}), flush=True)
 
 
+def run_router_only(args):
+    """The SoftTop-k router call alone on one workload (warmup + steps calls,
+    inputs resident). One JSON line; for profiling."""
+    import sparse_linear_attention_pool_b200 as sla
+
+    sla.load()
+    w = W.WORKLOADS[args.workload]
+    dev = device_inputs(W.make_inputs(w))
+    ms = time_router(sla, w, dev, args.steps, args.warmup)
+    print(json.dumps({"workload": w.name, "steps": args.steps, "warmup": args.warmup, "router_ms": round(ms, 4),
+                      "tau": ROUTER_TAU}), flush=True)
+
+
 def run_reference(args):
     """The oracle as it stands, timed on the host cores: one head per step."""
     rank = int(os.environ.get("RANK", "0"))
@@ -875,6 +889,8 @@ def main():
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--backward-only", action="store_true",
                     help="time sla_backward alone on --workload (one JSON line)")
+    ap.add_argument("--router-only", action="store_true",
+                    help="time sla_router_soft_topk alone on --workload (one JSON line)")
     ap.add_argument("--no-sla2-97", action="store_true",
                     help="skip the SLA2 97 %% entry (forward, router, backward)")
     ap.add_argument("--no-quant", action="store_true")
@@ -888,6 +904,8 @@ def main():
         run_sweep(args)
     elif args.backward_only:
         run_backward_only(args)
+    elif args.router_only:
+        run_router_only(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
