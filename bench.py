@@ -113,8 +113,9 @@ def attention_tile_bytes(w):
     step the K and V pairs, with phi(K)'s pair too when the excluded blocks'
     products run in phase 1 (d = 128 with a linear branch); per phase-2 step
     the phi(K) and V pairs (the negligible blocks, or at d = 64 every excluded
-    block); the phi(Q) pair when it is precomputed; SLA's W. None for the
-    quantised branch."""
+    block); the phi(Q) pair when it is precomputed; H_tot as a bf16 tile
+    (d = 128 with a linear branch) and SLA's W. None for the quantised
+    branch."""
     if w.precision != "bf16":
         return None
     tile = 64 * w.d * 2
@@ -127,6 +128,8 @@ def attention_tile_bytes(w):
     if pre:
         tiles += 2
     extra = w.d * w.d * 2 if (w.variant == "sla" and linear) else 0
+    if merged:
+        extra += w.d * w.d * 2
     ctas = w.B * w.H * ((w.Nb + 1) // 2)
     return ctas * (tiles * tile + extra)
 
@@ -244,7 +247,7 @@ def lowbit_peaks(bf16_burst):
 def stream_chunks(w):
     """Chunks per head of the K / V pass (one partial H and Z each): the
     streaming path (bf16, d = 128) sizes them for about 296 CTAs, the general
-    path takes 512 tokens per chunk."""
+    path (d = 64 or the quantised branch) takes 512 tokens per chunk."""
     if w.precision == "bf16" and w.d == 128:
         per_head = max(1, min(w.Nb, 296 // max(1, w.B * w.H)))
         cb = -(-w.Nb // per_head)
@@ -258,7 +261,9 @@ def stage_bytes(w):
     pool: Q read, pooled vectors written, phi(Q) written when the linear
     branch takes it precomputed; the general path (d = 64 or the quantised
     branch) reads K here too. phik_hz: K and V read, phi(K), z_j and the
-    chunks' partial H, Z written; the streaming path also writes the pooled K."""
+    chunks' partial H, Z written; the streaming path also writes the pooled K.
+    The quantised branch adds its codes (one byte per element of Q, K, V) and
+    block scales."""
     BH, N, Np, Nb, d = w.B * w.H, w.N, w.N_pad, w.Nb, w.d
     stream = w.precision == "bf16" and w.d == 128
     linear = w.k_crit + w.k_neg < Nb
@@ -270,6 +275,9 @@ def stage_bytes(w):
         kv += Nb * d * 4
     else:
         pool += N * d * 2 + Nb * d * 4
+    if w.precision != "bf16":  # Q and K codes in the pool pass, V codes in the K / V pass
+        pool += 2 * (Np * d + Nb * 4)
+        kv += Np * d + Nb * 4
     return {"pool": BH * pool, "phik_hz": BH * kv}
 
 

@@ -287,8 +287,17 @@ __global__ void __launch_bounds__(160, 3) q_stream_kernel(const __grid_constant_
           tma_store_3d(&maps.phiq, smem_u32(tile), 0, jb * kBlock, bh);
           tma_store_3d(&maps.phiq, smem_u32(tile) + kSub, 64, jb * kBlock, bh);
           bulk_commit();
-          bulk_wait_read<0>();
-          mbar_arrive(bar(kEmpty + s));
+          // the store of block j - 1 has read its stage: release that one
+          // (block j's is released one block later, so this block's store
+          // overlaps the next block's work)
+          if (j > 0) {
+            bulk_wait_read<1>();
+            mbar_arrive(bar(kEmpty + (j - 1) % kQStages));
+          }
+          if (j == nblk - 1) {
+            bulk_wait_read<0>();
+            mbar_arrive(bar(kEmpty + s));
+          }
         }
       } else {
         named_bar(1, 128);
@@ -503,11 +512,16 @@ cudaError_t launch_q_stream(const Layout& L, const __nv_bfloat16* Q, const __nv_
   memset(&maps, 0, sizeof(maps));
   if (!map_rows(&maps.q, Q, SD, L.N, L.Npad, L.BH)) return cudaErrorInvalidValue;
   if (phiq && !map_rows(&maps.phiq, phiq, SD, L.N, L.Npad, L.BH)) return cudaErrorInvalidValue;
-  QStreamArgs a{proj_q, qbar, status, L.N, L.Nb, L.stream_cb, phiq != nullptr ? 1 : 0, phi_elu1};
+  // the Q pass keeps no partial sums, so its chunks are sized on their own:
+  // about three CTAs per SM (its shared memory allows three)
+  const int per_head = std::max(1, std::min(L.Nb, 3 * (kStreamCtas / 2) / std::max(1, L.BH)));
+  const int cb = (L.Nb + per_head - 1) / per_head;
+  const int nchunk = (L.Nb + cb - 1) / cb;
+  QStreamArgs a{proj_q, qbar, status, L.N, L.Nb, cb, phiq != nullptr ? 1 : 0, phi_elu1};
   const int bytes = stream_smem_q();
   cudaError_t e = cudaFuncSetAttribute(q_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  q_stream_kernel<<<dim3(L.nchunk, L.BH), 160, bytes, s>>>(maps, a);
+  q_stream_kernel<<<dim3(nchunk, L.BH), 160, bytes, s>>>(maps, a);
   return cudaGetLastError();
 }
 

@@ -85,13 +85,13 @@ def test_job_value_counts_every_rank():
 def test_attention_tile_traffic_follows_the_load_schedule():
     # per CTA of two query blocks, in 16 KB tiles (64 rows x d = 128 bf16):
     # SLA 95 %: Q pair 2 + 25 critical steps x (K, V, phi(K) pairs) 6 + 51 negligible
-    # steps x (phi(K), V pairs) 4 + W (128 x 128 bf16 = 2 tiles) = 358
+    # steps x (phi(K), V pairs) 4 + W and H_tot (128 x 128 bf16 = 2 tiles each) = 360
     w = W.WORKLOADS["sla_wan13b_b1h12n32768d128_s95"]
     ctas = w.B * w.H * w.Nb // 2
-    assert bench.attention_tile_bytes(w) == ctas * 358 * 16384
-    # SLA2 97 %: Q pair 2 + 15 x 6 + the precomputed phi(Q) pair 2 = 94
+    assert bench.attention_tile_bytes(w) == ctas * 360 * 16384
+    # SLA2 97 %: Q pair 2 + 15 x 6 + the precomputed phi(Q) pair 2 + H_tot 2 = 96
     w2 = W.WORKLOADS["sla2_b1h12n32768d128_s97"]
-    assert bench.attention_tile_bytes(w2) == ctas * 94 * 16384
+    assert bench.attention_tile_bytes(w2) == ctas * 96 * 16384
     assert bench.attention_tile_bytes(W.WORKLOADS["sla2_q_wan14b_b1h40n75600d128_s97"]) is None
     f = bench.l2_fill(w, 1.0, {"sm_mhz": 1000.0}, 100)
     assert f["B_per_cycle_per_SM"] == pytest.approx(bench.attention_tile_bytes(w) / (1e-3 * 1e9 * 100), rel=1e-3)
