@@ -538,6 +538,33 @@ def time_backward(sla, w, dev, steps, warmup, dense=True):
     return bwd, fwd, dense
 
 
+def time_library_forward(w, dev, steps=5, warmup=2):
+    """ms per dense attention forward of the workload's shape through torch's
+    scaled_dot_product_attention, per backend (flash, cudnn): library kernels,
+    for context only; a backend that is unavailable is left out."""
+    import torch
+
+    out = {}
+    qd, kd, vd = (dev[x][:, :, :w.N] for x in ("q", "k", "v"))
+    for name, backend in (("flash", torch.nn.attention.SDPBackend.FLASH_ATTENTION),
+                          ("cudnn", torch.nn.attention.SDPBackend.CUDNN_ATTENTION)):
+        try:
+            with torch.nn.attention.sdpa_kernel(backend):
+                for _ in range(warmup):
+                    torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
+                start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                start.record()
+                for _ in range(steps):
+                    torch.nn.functional.scaled_dot_product_attention(qd, kd, vd)
+                end.record()
+                torch.cuda.synchronize()
+            out[name] = start.elapsed_time(end) / steps
+        except Exception:  # backend unavailable for this shape / build
+            pass
+    return out
+
+
 def time_router(sla, w, dev, steps, warmup, tau=ROUTER_TAU):
     """ms per SoftTop-k router call (pooling with the router projections, pooled
     scores, Pc and the per-row lambda / soft mask), on the current stream."""
@@ -699,6 +726,11 @@ def run_ours(args):
         res["dense_baseline"] = {"ms": round(dense_ms, 4),
                                  "tflops": round(dense_eq_flops(w) / (dense_ms * 1e-3) / 1e12, 2),
                                  "speedup_of_sparse": round(dense_ms / ms, 3)}
+        for name, fl in time_library_forward(w, dev).items():
+            res["dense_baseline"][f"library_{name}_forward"] = {
+                "ms": round(fl, 4), "tflops": round(dense_eq_flops(w) / (fl * 1e-3) / 1e12, 2),
+                "speedup_of_sparse": round(fl / ms, 3),
+                "note": f"torch scaled_dot_product_attention, {name} backend, same shape, for context"}
     if not args.no_sla2_97 and rank == 0 and args.workload != SLA2_97_WORKLOAD:
         w97 = W.WORKLOADS[SLA2_97_WORKLOAD]
         inp97 = W.make_inputs(w97)
@@ -716,7 +748,7 @@ def run_ours(args):
                  "executed_excl_masked_frac": round(useful_flops(w97) / t97 / 1e12 / pk97, 4),
                  "issued_tflops": round(executed_flops(w97) / t97 / 1e12, 2),
                  "peak": pk97, "peak_kind": pk97_kind, "traffic": ATTN_TRAFFIC.get(w97.name),
-                 "attention_l2_fill": fill97}
+                 "attention_l2_fill": fill97, "stages_ms": {k: round(v, 4) for k, v in st97.items()}}
         if "dense_baseline" in res:
             entry["speedup_vs_dense"] = round(res["dense_baseline"]["ms"] / ms97, 3)
         entry["router_soft_topk"] = {"ms": round(time_router(sla, w97, dev97, 20, 3), 4), "tau": ROUTER_TAU,
