@@ -154,7 +154,14 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   const bool merge = kMergeCapable && has_marg;
   // phi(Q) and Z_i precomputed (loaded) rather than formed in the epilogue
   const bool pre = has_marg && a.phiq != nullptr;
-  const int nP2 = has_marg ? (merge ? a.kn : nE) : 0;  // phase-2 ring steps
+  // quantised branch with a marginal set: phase 1's code tiles fill half of
+  // each ring slot, so every phase-1 step also carries one excluded block's
+  // phi(K) and V (bf16) in the other halves and its G product (block A's
+  // u-th excluded block on even steps, block B's on odd steps); phase 2 then
+  // takes the excluded blocks from index `carried` on
+  const bool hmerge = QNT && has_marg;
+  const int carried = hmerge ? nA / 2 : 0;
+  const int nP2 = has_marg ? (merge ? a.kn : nE - carried) : 0;  // phase-2 ring steps
   const int nTot = nA + nP2;                            // ring steps: phase 1 then phase 2
   const bool use_y = MODE == kModeSLA && a.w_proj != nullptr && has_marg;
   const int32_t* critA = a.crit + (size_t(bh) * Nb + iA) * a.kc;
@@ -181,7 +188,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
   auto step_block = [&](int X, int T) {
     if (dense) return T;
     if (T < nA) return checked((X ? critB : critA)[T]);
-    return excl_block(X, T - nA + (merge ? a.kc : 0));
+    return excl_block(X, T - nA + (merge ? a.kc : carried));
   };
   auto bar = [&](int b) { return smem_u32(&bars[b]); };
   auto wait = [&](int b, uint32_t parity) { return mbar_wait(bar(b), parity, abort_flag, a.status); };
@@ -305,6 +312,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
     constexpr int lag = C::kNK - C::kNV;  // K copies run this many steps ahead of V copies
     int kA_reg = 0, kB_reg = 0;           // indices of the current 32-step window (K side)
     int vA_reg = 0, vB_reg = 0;           // indices of the window the V side reads
+    int kH_reg = 0, vH_reg = 0;           // hmerge: the excluded block each phase-1 step carries
+    auto carried_block = [&](int T) { return excl_block(T & 1, T >> 1); };
     if (!merge) {
       for (int T = 0; T < nTot + lag && !stop; ++T) {
         const int TK = T, TV = T - lag;
@@ -312,23 +321,30 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           const int Ti = TK + lane;
           kA_reg = Ti < nTot ? step_block(0, Ti) : 0;
           kB_reg = Ti < nTot ? step_block(1, Ti) : 0;
+          kH_reg = Ti < 2 * carried ? carried_block(Ti) : 0;
         }
         if (TV >= 0 && (TV & 31) == 0 && TV < nTot) {
           const int Ti = TV + lane;
           vA_reg = Ti < nTot ? step_block(0, Ti) : 0;
           vB_reg = Ti < nTot ? step_block(1, Ti) : 0;
+          vH_reg = Ti < 2 * carried ? carried_block(Ti) : 0;
         }
         if (TK < nTot) {
           const int jA = __shfl_sync(0xffffffffu, kA_reg, TK & 31);
           const int jB = __shfl_sync(0xffffffffu, kB_reg, TK & 31);
+          const int jH = __shfl_sync(0xffffffffu, kH_reg, TK & 31);
           const int st = TK % C::kNK;
           if (!pwait(bKEmpty0 + st, ((TK / C::kNK) & 1) ^ 1)) break;
           if (lane == 0) {
             const uint32_t slot = sK + st * C::kPair;
             if (QNT && TK < nA) {
-              mbar_expect_tx(bar(bKFull0 + st), codeBytes);
+              const bool carry = TK < 2 * carried;
+              mbar_expect_tx(bar(bKFull0 + st), codeBytes + (carry ? C::kTile : 0));
               tma_load_3d(slot, &maps.kc, bar(bKFull0 + st), 0, jA * 64, bh);
               tma_load_3d(slot + C::kHalf, &maps.kc, bar(bKFull0 + st), 0, jB * 64, bh);
+              if (carry)  // phi(K) of the carried block in the slot's other half
+                for (int s = 0; s < C::kSub; ++s)
+                  tma_load_3d(slot + C::kSubS + s * 8192, &maps.phik, bar(bKFull0 + st), s * 64, jH * 64, bh);
             } else {
               const CUtensorMap* km = TK < nA ? &maps.k : &maps.phik;
               mbar_expect_tx(bar(bKFull0 + st), tileBytes);
@@ -345,14 +361,19 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         if (TV >= 0 && TV < nTot) {
           const int jA = __shfl_sync(0xffffffffu, vA_reg, TV & 31);
           const int jB = __shfl_sync(0xffffffffu, vB_reg, TV & 31);
+          const int jH = __shfl_sync(0xffffffffu, vH_reg, TV & 31);
           const int st = TV % C::kNV;
           if (!pwait(bVEmpty0 + st, ((TV / C::kNV) & 1) ^ 1)) break;
           if (lane == 0) {
             const uint32_t slot = sV + st * C::kPair;
             if (QNT && TV < nA) {
-              mbar_expect_tx(bar(bVFull0 + st), codeBytes);
+              const bool carry = TV < 2 * carried;
+              mbar_expect_tx(bar(bVFull0 + st), codeBytes + (carry ? C::kTile : 0));
               tma_load_3d(slot, &maps.vc, bar(bVFull0 + st), 0, jA * 64, bh);
               tma_load_3d(slot + C::kHalf, &maps.vc, bar(bVFull0 + st), 0, jB * 64, bh);
+              if (carry)  // V (bf16) of the carried block in the slot's other half
+                for (int s = 0; s < C::kSub; ++s)
+                  tma_load_3d(slot + C::kSubS + s * 8192, &maps.v, bar(bVFull0 + st), s * 64, jH * 64, bh);
             } else {
               mbar_expect_tx(bar(bVFull0 + st), tileBytes);
               for (int s = 0; s < C::kSub; ++s) {
@@ -488,6 +509,8 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
       constexpr uint32_t laneB = 16u << 16;  // D=64: G_B's M=64 accumulator starts at lane 16
       wait_w(bQFull, 0);
       tc_fence_after();
+      const uint32_t gA = tb + C::cG;
+      const uint32_t gB = D == 128 ? tb + C::cG + 128 : tb + laneB + C::cG;
       auto issue_pv = [&](int tp) {
         const int stv = tp % C::kNV;
         wait_w(bVFull0 + stv, (tp / C::kNV) & 1);
@@ -516,10 +539,22 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           }
         }
         mma_commit(bar(bPvDone));
+        if (hmerge) {
+          // the carried block's G += phi(K_j)^T V_j from the slots' other
+          // halves (64 tokens, M = N = D, MN-major, 64-column boxes 8 KB apart),
+          // then both slots are free
+          const int stk = tp % C::kNK;
+          if (tp < 2 * carried) {
+            const uint32_t kh = sK + stk * C::kPair + C::kSubS, vh = vslot + C::kSubS;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16((tp & 1) ? gB : gA, sdesc(kh + k * 2048, 8192, 1024), sdesc(vh + k * 2048, 8192, 1024),
+                       idesc_bf16(D, D, 1, 1), (tp >= 2 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(bKEmpty0 + stk));
+        }
         if (!merge) mma_commit(bar(bVEmpty0 + stv));  // merged: released after G
       };
-      const uint32_t gA = tb + C::cG;
-      const uint32_t gB = D == 128 ? tb + C::cG + 128 : tb + laneB + C::cG;
       // G += phi(K_j)^T V_j for both blocks (M = N = D, MN-major operands; the
       // j_B rows sit kHalf into each sub-tile)
       auto issue_g = [&](uint32_t kslot, uint32_t vslot, bool first) {
@@ -567,7 +602,9 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
           }
         }
         mma_commit(bar(bSFull));
-        mma_commit(bar(merge ? bKDone0 + stk : bKEmpty0 + stk));  // merged: phi(K) refills the slot
+        // merged: phi(K) refills the slot; hmerge: the slot is released after
+        // the carried block's G, with its PV
+        if (!hmerge) mma_commit(bar(merge ? bKDone0 + stk : bKEmpty0 + stk));
         if (pre && t == nA - 1) mma_commit(bar(bQFree));          // Q tiles free for phi(Q)
         if (t > 0) {
           issue_pv(t - 1);
@@ -583,7 +620,7 @@ __global__ void __launch_bounds__(192, 1) attn_tc_kernel(const __grid_constant__
         wait_kfull(stk);
         wait_w(bVFull0 + stv, (T / C::kNV) & 1);
         tc_fence_after();
-        issue_g(sK + stk * C::kPair, sV + stv * C::kPair, !merge && u == 0);
+        issue_g(sK + stk * C::kPair, sV + stv * C::kPair, !merge && carried == 0 && u == 0);
         mma_commit(bar(bKEmpty0 + stk));
         mma_commit(bar(bVEmpty0 + stv));
       }
