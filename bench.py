@@ -661,6 +661,8 @@ def run_ours(args):
     sla.load()
     pk, pk_kind = peaks()
     w = W.WORKLOADS[args.workload]
+    if args.heads:  # a slice of the workload's heads (profiler captures); the name says so
+        w = w.replace(H=args.heads, name=f"{w.name}_h{args.heads}")
     inp = W.make_inputs(w)
     dev = device_inputs(inp)
     clocks = ClockSampler(local)
@@ -836,6 +838,10 @@ def run_sweep(args):
         dms = time_dense(sla, base, dev, dense_steps, 2)
         rows.append({"N": N, "variant": "dense", "sparsity": 0, "ms": round(dms, 4),
                      "dense_eq_tflops": round(dense_eq_flops(base) / (dms * 1e-3) / 1e12, 1)})
+        # torch's dense attention on the same inputs, for context
+        for name, lms in time_library_forward(base, dev, steps=dense_steps).items():
+            rows.append({"N": N, "variant": f"library_{name}", "sparsity": 0, "ms": round(lms, 4),
+                         "dense_eq_tflops": round(dense_eq_flops(base) / (lms * 1e-3) / 1e12, 1)})
         for variant in ("sla", "sla2"):
             for sp in SWEEP_SPARSITY:
                 w = W.sweep_workload(N, sp, variant)
@@ -924,6 +930,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only this many heads of the workload (for profiler captures)")
     ap.add_argument("--dense-steps", type=int, default=5)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
